@@ -1,0 +1,213 @@
+// C ABI of the AWQ W4A16 library: argument checks, launch configuration, and the
+// entry points declared in include/awq.h.  The whole library is one translation
+// unit (this file includes the kernel headers), so the device error word and the
+// kernels share one module.
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemv.cuh"
+#include "quantize.cuh"
+#include "gemm_sm100.cuh"
+#include "search.cuh"
+
+using namespace awq;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int max_smem_optin = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+bool device_info(DeviceInfo& out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+        if (cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+            return false;
+        d.ready = true;
+    }
+    out = d;
+    return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+awq_status check_config(const awq_quant_config& c) {
+    if (c.zero_point != 0 && c.zero_point != 1) return AWQ_ERR_INVALID_ARG;
+    if (c.w_bit != 4) return AWQ_ERR_UNSUPPORTED;
+    if (c.q_group_size != 32 && c.q_group_size != 64 && c.q_group_size != 128 && c.q_group_size != 256)
+        return AWQ_ERR_UNSUPPORTED;
+    return AWQ_OK;
+}
+
+awq_status check_shape(int N, int K, const awq_quant_config& c) {
+    if (N <= 0 || K <= 0) return AWQ_ERR_INVALID_ARG;
+    if (K % c.q_group_size != 0) return AWQ_ERR_INVALID_ARG;
+    return AWQ_OK;
+}
+
+awq_status launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+// Checks shared by the two linear entry points.
+awq_status check_linear(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
+                        const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg,
+                        const uint16_t* Y) {
+    awq_status st = check_config(cfg);
+    if (st != AWQ_OK) return st;
+    st = check_shape(N, K, cfg);
+    if (st != AWQ_OK) return st;
+    if (M <= 0) return AWQ_ERR_INVALID_ARG;
+    if (!X || !qweight || !scales || !Y) return AWQ_ERR_INVALID_ARG;
+    if (cfg.zero_point && !qzeros) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(Y)) return AWQ_ERR_INVALID_ARG;
+    if (qzeros && !aligned16(qzeros)) return AWQ_ERR_INVALID_ARG;
+    return AWQ_OK;
+}
+
+template <int MT>
+awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
+                       const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
+                       cudaStream_t st) {
+    constexpr int R = gemv_rows_per_warp(MT);
+    DeviceInfo d;
+    if (!device_info(d)) return AWQ_ERR_CUDA;
+    const size_t smem = gemv_smem_bytes(MT, K);
+    if (smem > (size_t)d.max_smem_optin) return AWQ_ERR_UNSUPPORTED;
+    auto kern = gemv_kernel<MT, R>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return AWQ_ERR_CUDA;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvThreads, smem) != cudaSuccess || occ < 1)
+        return AWQ_ERR_CUDA;
+    const int row_groups = ceil_div(N, R);
+    const int want = ceil_div(row_groups, kGemvWarps);
+    const int grid = want < d.sms * occ ? want : d.sms * occ;
+    kern<<<grid, kGemvThreads, smem, st>>>(X, M, qweight, scales, qzeros, N, K, cfg.q_group_size,
+                                           cfg.zero_point, Y);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* awq_status_string(awq_status s) {
+    switch (s) {
+        case AWQ_OK: return "AWQ_OK";
+        case AWQ_ERR_INVALID_ARG: return "AWQ_ERR_INVALID_ARG: invalid argument (null/misaligned pointer or bad size)";
+        case AWQ_ERR_UNSUPPORTED: return "AWQ_ERR_UNSUPPORTED: configuration not supported";
+        case AWQ_ERR_WORKSPACE: return "AWQ_ERR_WORKSPACE: workspace too small";
+        case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA: a CUDA call or kernel launch failed";
+        case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT: a bounded device wait ran out";
+    }
+    return "AWQ_ERR_UNKNOWN";
+}
+
+int32_t awq_abi_version(void) { return 1; }
+
+awq_status awq_quantize_pack(const uint16_t* W, const uint16_t* s, int32_t N, int32_t K, awq_quant_config cfg,
+                             uint32_t* qweight, uint16_t* scales, uint32_t* qzeros, void* stream) {
+    awq_status st = check_config(cfg);
+    if (st != AWQ_OK) return st;
+    st = check_shape(N, K, cfg);
+    if (st != AWQ_OK) return st;
+    if (!W || !qweight || !scales) return AWQ_ERR_INVALID_ARG;
+    if (cfg.zero_point && !qzeros) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(qweight) || (s && !aligned16(s))) return AWQ_ERR_INVALID_ARG;
+    const long long blocks = (long long)N * ceil_div(K, kQuantChunk);
+    if (blocks > 0x7fffffffLL) return AWQ_ERR_UNSUPPORTED;
+    quantize_pack_kernel<<<(unsigned)blocks, kQuantThreads, 0, (cudaStream_t)stream>>>(
+        W, s, N, K, cfg.q_group_size, cfg.zero_point, qweight, scales, cfg.zero_point ? qzeros : nullptr);
+    return launch_status();
+}
+
+awq_status awq_fold_inverse_scale(const uint16_t* X, const uint16_t* s, int32_t M, int32_t K, uint16_t* X_out,
+                                  void* stream) {
+    if (!X || !s || !X_out || M <= 0 || K <= 0 || (K & 7)) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(s) || !aligned16(X_out)) return AWQ_ERR_INVALID_ARG;
+    DeviceInfo d;
+    if (!device_info(d)) return AWQ_ERR_CUDA;
+    const long long units = (long long)M * K / 8;
+    long long grid = (units + 255) / 256;
+    if (grid > 8LL * d.sms) grid = 8LL * d.sms;
+    fold_inverse_scale_kernel<<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(X, s, M, K, X_out);
+    return launch_status();
+}
+
+awq_status awq_linear_gemv(const uint16_t* X, int32_t M, const uint32_t* qweight, const uint16_t* scales,
+                           const uint32_t* qzeros, int32_t N, int32_t K, awq_quant_config cfg, uint16_t* Y,
+                           void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    awq_status st = check_linear(X, M, qweight, scales, qzeros, N, K, cfg, Y);
+    if (st != AWQ_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (M == 1) return launch_gemv<1>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+    if (M == 2) return launch_gemv<2>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+    if (M <= 4) return launch_gemv<4>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+    if (M <= 8) return launch_gemv<8>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+    return AWQ_ERR_UNSUPPORTED;
+}
+
+awq_status awq_linear_gemm(const uint16_t* X, int32_t M, const uint32_t* qweight, const uint16_t* scales,
+                           const uint32_t* qzeros, int32_t N, int32_t K, awq_quant_config cfg, uint16_t* Y,
+                           void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    awq_status st = check_linear(X, M, qweight, scales, qzeros, N, K, cfg, Y);
+    if (st != AWQ_OK) return st;
+    DeviceInfo d;
+    if (!device_info(d)) return AWQ_ERR_CUDA;
+    return launch_gemm_w4a16(X, M, qweight, scales, qzeros, N, K, cfg.q_group_size, cfg.zero_point, Y,
+                             (cudaStream_t)stream, d.sms);
+}
+
+size_t awq_workspace_bytes(int32_t op, int32_t M, int32_t N, int32_t K, awq_quant_config cfg) {
+    if (op == AWQ_OP_SCALE_SEARCH) return search_workspace_bytes(M, N, K, cfg.q_group_size, 64);
+    return 0;
+}
+
+awq_status awq_scale_search(const uint16_t* X, int32_t M, const uint16_t* W, int32_t N, int32_t K,
+                            awq_quant_config cfg, int32_t n_grid, uint16_t* s_out, double* losses_out,
+                            int32_t* best_index_out, void* ws, size_t ws_bytes, void* stream) {
+    awq_status st = check_config(cfg);
+    if (st != AWQ_OK) return st;
+    st = check_shape(N, K, cfg);
+    if (st != AWQ_OK) return st;
+    if (M <= 0 || n_grid < 1 || n_grid > 64) return AWQ_ERR_INVALID_ARG;
+    if (!X || !W || !s_out || !ws) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(s_out) || !aligned16(ws)) return AWQ_ERR_INVALID_ARG;
+    if (ws_bytes < search_workspace_bytes(M, N, K, cfg.q_group_size, n_grid)) return AWQ_ERR_WORKSPACE;
+    DeviceInfo d;
+    if (!device_info(d)) return AWQ_ERR_CUDA;
+    return run_scale_search(X, M, W, N, K, cfg.q_group_size, cfg.zero_point, n_grid, s_out, losses_out,
+                            best_index_out, ws, (cudaStream_t)stream, d.sms);
+}
+
+awq_status awq_device_error(void* stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return AWQ_ERR_CUDA;
+    unsigned word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return AWQ_ERR_CUDA;
+    if (word == 0) return AWQ_OK;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return AWQ_ERR_CUDA;
+    return AWQ_ERR_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,48 @@
+// Shared device helpers of the AWQ W4A16 library (sm_100a).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "awq.h"
+
+namespace awq {
+
+// Bit set in the device error word when a bounded wait runs out.
+constexpr unsigned kErrTimeout = 1u;
+
+// One error word per device that loads the library.  Kernels OR flags into it;
+// awq_device_error() reads and clears it.
+__device__ unsigned int g_error_word;
+
+__device__ __forceinline__ void raise_error(unsigned flag) { atomicOr(&g_error_word, flag); }
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait limit for every spin in this library: 2 s of wall time.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// ---------------------------------------------------------------------------
+// fp16 helpers (bit patterns in, bit patterns out)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+__device__ __forceinline__ uint16_t f2h_rn(float f) { return __half_as_ushort(__float2half_rn(f)); }
+
+// Correctly rounded double -> binary16 (one rounding, nearest-even), by the
+// PTX conversion instruction.
+__device__ __forceinline__ uint16_t d2h_rn(double d) {
+    uint16_t h;
+    asm("cvt.rn.f16.f64 %0, %1;" : "=h"(h) : "d"(d));
+    return h;
+}
+
+__host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace awq

@@ -1,0 +1,306 @@
+// Fused dequantising W4A16 GEMM on the sm_100a tensor cores (tcgen05 + TMA + TMEM).
+//
+// Source: "Optimization Awq" (skillsdirectory.com), kernel backends: GEMM is the
+// default for batch sizes > 1 (batched decode and prefill); "AI-Research-SKILLs AWQ
+// advanced usage guide" (lshu.cn), WQLinear kernels.  Result as the header defines:
+// Y[m][n] = sum_k X[m][k] * (q[n][k] - z[n][g]) * scale16[n][g], fp32 accumulation.
+//
+// Formulation.  The kernel computes Y^T tile by tile: D[n][m] = sum_k Wdeq[n][k] X[m][k]
+// with the dequantised weight tile as the MMA's A operand (M_mma = 128 output
+// channels) and the activations as B (N_mma = BN tokens, 16..256).  Each weight tile
+// is dequantised once per CTA and reused for BN tokens, so the dequant work per
+// multiply-add is 1/BN, and small token counts use a narrow MMA instead of padding.
+//
+// Warp roles (320 threads):
+//   warp 0      TMA producer: X tile [BN x 64] fp16 (128B swizzle) and the packed
+//               weight tile [128 x 8 words] per 64-channel k-block, into an S-stage ring.
+//   warp 1      allocates TMEM; one lane issues 4 tcgen05.mma (K = 16 each) per k-block.
+//   warps 2..9  dequantise: thread (row, half) turns 32 codes into fp16
+//               (q - z) * scale16 with mask/magic-number arithmetic and writes them in
+//               the 128B-swizzled K-major layout the MMA reads; afterwards they are the
+//               epilogue, reading the fp32 accumulator from TMEM and storing fp16 Y.
+// Every wait is bounded (2 s): on time-out the kernel raises the device error word,
+// drains what it issued, frees TMEM and returns.
+#pragma once
+
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace awq {
+
+constexpr int kGemmThreads = 320;
+constexpr int kGemmTileN = 128;      // output channels per CTA (MMA M)
+constexpr int kGemmKB = 64;          // input channels per k-block
+constexpr int kDequantThreads = 256;
+
+template <int BN>
+struct GemmCfg {
+    static constexpr int kStages = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
+    static constexpr int kABufs = BN >= 256 ? 3 : 4;
+    static constexpr int kXBytes = BN * 128;                 // X tile: BN rows x 128 B
+    static constexpr int kWBytes = kGemmTileN * 32;          // packed tile: 128 rows x 32 B
+    static constexpr int kABytes = kGemmTileN * 128;         // dequantised tile
+    static constexpr int kXOff = 0;
+    static constexpr int kAOff = kXOff + kStages * kXBytes;  // both multiples of 1024
+    static constexpr int kWOff = kAOff + kABufs * kABytes;
+    static constexpr int kBarOff = kWOff + kStages * kWBytes;
+    static constexpr int kNumBars = 2 * kStages + 2 * kABufs + 1;
+    static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kTmemPtrOff + 16 + 1024;   // + slack to align the base to 1024
+    static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+};
+
+// (q - z) * s for the 8 codes of one word, returned as 4 fp16 pairs in k order.
+__device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t zmagic, uint32_t zneg16, uint32_t s2) {
+    const uint32_t kMagic = 0x64006400u;     // fp16 1024 in both halves
+    const uint32_t kSixteenth = 0x2C002C00u; // fp16 1/16 in both halves
+    uint32_t a = (w & 0x000F000Fu) | kMagic;            // 1024 + q0, 1024 + q4
+    uint32_t b = (w & 0x00F000F0u) | kMagic;            // 1024 + 16 q1, 1024 + 16 q5
+    const uint32_t w8 = w >> 8;
+    uint32_t c = (w8 & 0x000F000Fu) | kMagic;           // q2, q6
+    uint32_t d = (w8 & 0x00F000F0u) | kMagic;           // q3, q7
+    asm("sub.rn.f16x2 %0, %0, %4;\n\t"                  // q - z (exact)
+        "fma.rn.f16x2 %1, %1, %5, %6;\n\t"              // (1024 + 16q)/16 - (64 + z) = q - z (exact)
+        "sub.rn.f16x2 %2, %2, %4;\n\t"
+        "fma.rn.f16x2 %3, %3, %5, %6;\n\t"
+        "mul.rn.f16x2 %0, %0, %7;\n\t"                  // * scale16 (one rounding)
+        "mul.rn.f16x2 %1, %1, %7;\n\t"
+        "mul.rn.f16x2 %2, %2, %7;\n\t"
+        "mul.rn.f16x2 %3, %3, %7;"
+        : "+r"(a), "+r"(b), "+r"(c), "+r"(d)
+        : "r"(zmagic), "r"(kSixteenth), "r"(zneg16), "r"(s2));
+    uint4 o;
+    o.x = __byte_perm(a, b, 0x5410);   // (k0, k1)
+    o.y = __byte_perm(c, d, 0x5410);   // (k2, k3)
+    o.z = __byte_perm(a, b, 0x7632);   // (k4, k5)
+    o.w = __byte_perm(c, d, 0x7632);   // (k6, k7)
+    return o;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
+                  const uint16_t* __restrict__ scales, const uint32_t* __restrict__ qzeros, int M, int N, int K,
+                  int G, int zero_point, uint16_t* __restrict__ Y) {
+    using C = GemmCfg<BN>;
+    using namespace sm100;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    uint64_t* full = bars;                          // [kStages]  TMA landed
+    uint64_t* empty = bars + C::kStages;            // [kStages]  MMA done with the X / packed slot
+    uint64_t* afull = empty + C::kStages;           // [kABufs]   dequantised tile written
+    uint64_t* aempty = afull + C::kABufs;           // [kABufs]   MMA done with the dequantised tile
+    uint64_t* tfull = aempty + C::kABufs;           // accumulator complete
+    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::kTmemPtrOff);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * BN;
+    const int n0 = blockIdx.y * kGemmTileN;
+    const int num_kb = ceil_div(K, kGemmKB);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < C::kABufs; ++a) {
+            mbar_init(&afull[a], kDequantThreads / 32);
+            mbar_init(&aempty[a], 1);
+        }
+        mbar_init(tfull, 1);
+        mbar_fence_init();
+        prefetch_tensormap(&tmap_x);
+        prefetch_tensormap(&tmap_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_ptr, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            int issued = 0;
+            bool ok = true;
+            for (int kb = 0; kb < num_kb && ok; ++kb) {
+                const int s = kb % C::kStages;
+                if (kb >= C::kStages) ok = mbar_wait(&empty[s], ((kb / C::kStages) - 1) & 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&full[s], C::kXBytes + C::kWBytes);
+                tma_load_2d(smem + C::kXOff + s * C::kXBytes, &tmap_x, &full[s], kb * kGemmKB, m0);
+                tma_load_2d(smem + C::kWOff + s * C::kWBytes, &tmap_q, &full[s], kb * (kGemmKB / 8), n0);
+                ++issued;
+            }
+            // Drain: every issued copy must land before the CTA may exit.
+            for (int kb = issued - 1; kb >= 0 && kb >= issued - C::kStages; --kb)
+                mbar_wait(&full[kb % C::kStages], (kb / C::kStages) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            constexpr uint32_t idesc = idesc_f16_f32(kGemmTileN, BN);
+            bool ok = true;
+            for (int kb = 0; kb < num_kb && ok; ++kb) {
+                const int s = kb % C::kStages;
+                const int a = kb % C::kABufs;
+                ok = mbar_wait(&full[s], (kb / C::kStages) & 1) && mbar_wait(&afull[a], (kb / C::kABufs) & 1);
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t adesc = desc_sw128_kmajor(smem_u32(smem + C::kAOff + a * C::kABytes));
+                const uint64_t bdesc = desc_sw128_kmajor(smem_u32(smem + C::kXOff + s * C::kXBytes));
+#pragma unroll
+                for (int kk = 0; kk < kGemmKB / 16; ++kk)
+                    mma_f16(tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+                mma_commit(&empty[s]);
+                mma_commit(&aempty[a]);
+            }
+            mma_commit(tfull);   // also on the error path, so that the MMAs drain before TMEM is freed
+            if (!ok) mbar_wait(tfull, 0);
+        }
+    } else {
+        // ---------------- dequantise, then epilogue ----------------
+        const int d = threadIdx.x - 64;           // 0..255
+        const int row = d & (kGemmTileN - 1);
+        const int kh = d >> 7;                    // which 32 channels of the k-block
+        const int n = n0 + row;
+        const int ng = K / G;
+        const int nzw = ceil_div(ng, 8);
+        const bool zp = zero_point != 0;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb && ok; ++kb) {
+            const int s = kb % C::kStages;
+            const int a = kb % C::kABufs;
+            const int k = kb * kGemmKB + kh * 32;
+            // scale / zero of this thread's 32 channels (one group: G >= 32)
+            uint32_t s2 = 0, zmagic = 0x64006400u, zneg16 = 0;
+            const bool live = n < N && k < K;
+            if (live) {
+                const int g = k / G;
+                const uint32_t sc = __ldg(scales + (size_t)n * ng + g);
+                const uint32_t z = zp ? ((__ldg(qzeros + (size_t)n * nzw + (g >> 3)) >> (4 * (g & 7))) & 15u) : 8u;
+                s2 = sc | (sc << 16);
+                const uint32_t zm = 0x6400u | z;                                   // 1024 + z
+                zmagic = zm | (zm << 16);
+                const uint32_t zn = __half_as_ushort(__float2half_rn(-(64.0f + (float)z)));
+                zneg16 = zn | (zn << 16);
+            }
+            if (kb >= C::kABufs) ok = mbar_wait(&aempty[a], ((kb / C::kABufs) - 1) & 1);
+            ok = ok && mbar_wait(&full[s], (kb / C::kStages) & 1);
+            if (!ok) break;
+            const uint4 packed =
+                *reinterpret_cast<const uint4*>(smem + C::kWOff + s * C::kWBytes + row * 32 + kh * 16);
+            uint8_t* atile = smem + C::kAOff + a * C::kABytes;
+            const uint32_t pw[4] = {packed.x, packed.y, packed.z, packed.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 v = live ? dequant_word(pw[i], zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(atile + sw128_offset(row, kh * 4 + i)) = v;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[a]);
+        }
+        if (ok && mbar_wait(tfull, 0)) {
+            tc_fence_after();
+            const int q = warp & 3;                        // TMEM lane quarter this warp may access
+            const int set = (warp - 2) >> 2;               // 0: warps 2..5, 1: warps 6..9
+            const int cols = BN >= 32 ? BN / 2 : BN;
+            const int c_begin = BN >= 32 ? set * cols : 0;
+            if (BN >= 32 || set == 0) {
+                const int nn = n0 + q * 32 + lane;
+                for (int c = c_begin; c < c_begin + cols; c += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, r);
+                    tmem_ld_wait();
+                    if (nn < N) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int m = m0 + c + j;
+                            if (m < M) Y[(size_t)m * N + nn] = f2h_rn(__uint_as_float(r[j]));
+                        }
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [rows][cols] of `esize`-byte elements; box [box_rows][box_cols].
+inline bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int esize, uint64_t rows,
+                         uint64_t cols, uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swz) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)esize};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN>
+awq_status launch_gemm_bn(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
+                          const uint32_t* qzeros, int N, int K, int G, int zp, uint16_t* Y, cudaStream_t st) {
+    using C = GemmCfg<BN>;
+    CUtensorMap tx, tq;
+    if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)M, (uint64_t)K, BN, kGemmKB,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return AWQ_ERR_CUDA;
+    if (!make_tmap_2d(&tq, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)N, (uint64_t)(K / 8), kGemmTileN,
+                      kGemmKB / 8, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return AWQ_ERR_CUDA;
+    auto kern = gemm_w4a16_kernel<BN>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return AWQ_ERR_CUDA;
+    dim3 grid(ceil_div(M, BN), ceil_div(N, kGemmTileN));
+    if (grid.y > 65535u) return AWQ_ERR_UNSUPPORTED;
+    kern<<<grid, kGemmThreads, C::kSmemBytes, st>>>(tx, tq, scales, qzeros, M, N, K, G, zp, Y);
+    return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+inline awq_status launch_gemm_w4a16(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
+                                    const uint32_t* qzeros, int N, int K, int G, int zp, uint16_t* Y, cudaStream_t st,
+                                    int /*sms*/) {
+    if (M <= 16) return launch_gemm_bn<16>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
+    if (M <= 32) return launch_gemm_bn<32>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
+    if (M <= 64) return launch_gemm_bn<64>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
+    if (M <= 128) return launch_gemm_bn<128>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
+    return launch_gemm_bn<256>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
+}
+
+}  // namespace awq

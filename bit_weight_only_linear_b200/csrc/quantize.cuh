@@ -1,0 +1,188 @@
+// Group quantise + pack, activation statistic, alpha -> s, and the activation fold.
+//
+// Source of the arithmetic: "AI-Research-SKILLs AWQ advanced usage guide"
+// (lshu.cn), sections 算法原理 (scale s from activation statistics, W*s quantised,
+// s^-1 folded into X) and 量化超参数调优 (group size; zero-point = offset for
+// asymmetric ranges, off = symmetric), with the quantiser the library fixes:
+// scale = (max-min)/15 or max|w|/7, zero = clamp(rint(-min/scale), 0, 15),
+// q = clamp(rint(w/scale) + zero, 0, 15), all IEEE fp32, round-half-even.
+#pragma once
+
+#include "common.cuh"
+
+namespace awq {
+
+constexpr int kQuantThreads = 256;                 // 8 elements per thread
+constexpr int kQuantChunk = kQuantThreads * 8;     // 2048 input channels per block
+constexpr float kScaleFloor = 1e-5f;
+
+struct GroupParams {
+    float sc;     // fp32 value of the fp16 scale
+    float zero;   // integer-valued
+    uint16_t sc16;
+};
+
+// Per-group scale/zero from the group's extreme values, as the header defines.
+__device__ __forceinline__ GroupParams group_params(float mx, float mn, bool zero_point) {
+    GroupParams p;
+    if (zero_point) {
+        float scale32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+        scale32 = fmaxf(scale32, kScaleFloor);
+        p.sc16 = f2h_rn(scale32);
+        p.sc = h2f(p.sc16);
+        p.zero = fminf(fmaxf(rintf(__fdiv_rn(-mn, p.sc)), 0.0f), 15.0f);
+    } else {
+        float amax = fmaxf(fabsf(mx), fabsf(mn));
+        float scale32 = __fdiv_rn(amax, 7.0f);
+        scale32 = fmaxf(scale32, kScaleFloor);
+        p.sc16 = f2h_rn(scale32);
+        p.sc = h2f(p.sc16);
+        p.zero = 8.0f;
+    }
+    return p;
+}
+
+// Code of one scaled weight.
+__device__ __forceinline__ uint32_t quant_code(float ws, const GroupParams& p, bool zero_point) {
+    float r = rintf(__fdiv_rn(ws, p.sc));
+    if (zero_point) return (uint32_t)fminf(fmaxf(r + p.zero, 0.0f), 15.0f);
+    return (uint32_t)(fminf(fmaxf(r, -8.0f), 7.0f) + 8.0f);
+}
+
+// Butterfly max/min over the `seg` consecutive lanes (power of two) that hold a group.
+__device__ __forceinline__ void seg_minmax(float& mx, float& mn, int seg) {
+    for (int off = seg >> 1; off > 0; off >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    }
+}
+
+// One block per (row, 2048-channel chunk); thread t owns channels [8t, 8t+8) of the
+// chunk and writes one qweight word.  A group of G channels spans G/8 lanes of one
+// warp, so its min/max is a shuffle butterfly; the chunk holds whole zero words
+// (2048/G groups, a multiple of 8), packed through shared memory.
+__global__ void __launch_bounds__(kQuantThreads)
+quantize_pack_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict__ s, int N, int K,
+                     int G, int zero_point, uint32_t* __restrict__ qweight,
+                     uint16_t* __restrict__ scales, uint32_t* __restrict__ qzeros) {
+    __shared__ uint8_t zbuf[kQuantChunk / 32];
+    const int nchunks = ceil_div(K, kQuantChunk);
+    const int row = blockIdx.x / nchunks;
+    const int chunk = blockIdx.x % nchunks;
+    const int k0 = chunk * kQuantChunk + threadIdx.x * 8;
+    const bool active = k0 < K;
+    const bool zp = zero_point != 0;
+
+    float ws[8];
+    if (active) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(W + (size_t)row * K + k0);
+        const uint16_t* wh = reinterpret_cast<const uint16_t*>(&wv);
+        if (s != nullptr) {
+            const uint4 sv = *reinterpret_cast<const uint4*>(s + k0);
+            const uint16_t* sh = reinterpret_cast<const uint16_t*>(&sv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ws[i] = __fmul_rn(h2f(wh[i]), h2f(sh[i]));   // exact
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ws[i] = h2f(wh[i]);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ws[i] = 0.0f;
+    }
+    float mx = ws[0], mn = ws[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+        mx = fmaxf(mx, ws[i]);
+        mn = fminf(mn, ws[i]);
+    }
+    seg_minmax(mx, mn, G >> 3);
+    const GroupParams p = group_params(mx, mn, zp);
+
+    const int ng = K / G;
+    if (active) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) word |= quant_code(ws[i], p, zp) << (4 * i);
+        qweight[(size_t)row * (K >> 3) + (k0 >> 3)] = word;
+        if ((k0 % G) == 0) {
+            const int g = k0 / G;
+            scales[(size_t)row * ng + g] = p.sc16;
+            zbuf[(threadIdx.x * 8) / G] = (uint8_t)p.zero;
+        }
+    }
+    if (!zp) return;
+    __syncthreads();
+    const int groups_here = kQuantChunk / G;          // multiple of 8
+    const int g_base = chunk * groups_here;
+    const int zw = threadIdx.x;
+    if (zw < groups_here / 8 && g_base + zw * 8 < ng) {
+        uint32_t word = 0;
+        for (int i = 0; i < 8; ++i) {
+            const int g = g_base + zw * 8 + i;
+            if (g < ng) word |= (uint32_t)zbuf[zw * 8 + i] << (4 * i);
+        }
+        qzeros[(size_t)row * ceil_div(ng, 8) + (g_base >> 3) + zw] = word;
+    }
+}
+
+// Column sums of |X| in fp64.  Every partial sum is an exact fp64 number (fp16
+// values are multiples of 2^-24 and the sums stay far below 2^29), so the atomic
+// accumulation is exact and order-independent.  Block: 128 threads x 8 columns;
+// grid.y splits the rows.
+__global__ void __launch_bounds__(128)
+abs_colsum_kernel(const uint16_t* __restrict__ X, int M, int K, double* __restrict__ colsum) {
+    const int c0 = (blockIdx.x * 128 + threadIdx.x) * 8;
+    if (c0 >= K) return;
+    const int rows_per = ceil_div(M, gridDim.y);
+    const int r0 = blockIdx.y * rows_per;
+    const int r1 = min(M, r0 + rows_per);
+    double acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+    for (int r = r0; r < r1; ++r) {
+        const uint4 v = *reinterpret_cast<const uint4*>(X + (size_t)r * K + c0);
+        const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += (double)fabsf(h2f(h[i]));
+    }
+    if (r1 > r0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) atomicAdd(colsum + c0 + i, acc[i]);
+    }
+}
+
+// s[a][k] = fp16(max(pow(colsum[k]/M, a/n_grid), 2^-14)) for every alpha of the grid.
+__global__ void scales_for_alphas_kernel(const double* __restrict__ colsum, int M, int K,
+                                         int n_grid, uint16_t* __restrict__ s_all) {
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    const int a = blockIdx.y;
+    if (k >= K) return;
+    const double m = __ddiv_rn(colsum[k], (double)M);
+    const double alpha = __ddiv_rn((double)a, (double)n_grid);
+    double p = pow(m, alpha);
+    p = fmax(p, 6.103515625e-05);   // 2^-14
+    s_all[(size_t)a * K + k] = d2h_rn(p);
+}
+
+// X_out = fp16(fp32(X) / fp32(s)), 8 elements per thread, grid-stride.
+__global__ void fold_inverse_scale_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ s,
+                                          int M, int K, uint16_t* __restrict__ Xo) {
+    const size_t total8 = (size_t)M * K / 8;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total8;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const size_t e = i * 8;
+        const int k = (int)(e % K);
+        const uint4 xv = *reinterpret_cast<const uint4*>(X + e);
+        const uint4 sv = *reinterpret_cast<const uint4*>(s + k);
+        const uint16_t* xh = reinterpret_cast<const uint16_t*>(&xv);
+        const uint16_t* sh = reinterpret_cast<const uint16_t*>(&sv);
+        uint4 ov;
+        uint16_t* oh = reinterpret_cast<uint16_t*>(&ov);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) oh[j] = f2h_rn(__fdiv_rn(h2f(xh[j]), h2f(sh[j])));
+        *reinterpret_cast<uint4*>(Xo + e) = ov;
+    }
+}
+
+}  // namespace awq

@@ -1,0 +1,168 @@
+/*
+ * awq.h - C ABI of the B200 (sm_100a) AWQ group-wise W4A16 library.
+ *
+ * The operations are the per-layer core of activation-aware weight quantisation
+ * (AWQ) as the pages describe it:
+ *   - "AI-Research-SKILLs AWQ advanced usage guide" (lshu.cn), section 算法原理:
+ *     the objective L(s) = || Q(W*s)(s^-1*X) - W*X || over a per-input-channel
+ *     scale s derived from activation statistics; salient channels are protected
+ *     by scaling, with no mixed precision;
+ *   - same page, section 量化超参数调优 (group size and zero-point choices) and
+ *     section "WQLinear kernels" (GEMM for batches, GEMV for a single token);
+ *   - "Optimization Awq" (skillsdirectory.com), the quant_config block
+ *     {"zero_point", "q_group_size", "w_bit": 4, "version": "GEMM" | "GEMV"}.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Types.    fp16 tensors are passed as `uint16_t*` holding IEEE binary16 bit
+ *           patterns; packed codes as `uint32_t*`.  No CUDA or framework type
+ *           appears in a signature: `stream` is a `cudaStream_t` passed as
+ *           `void*` (NULL = the legacy default stream).
+ * Memory.   Every tensor pointer is DEVICE memory owned by the caller unless the
+ *           argument says "host".  The library never allocates, frees or keeps a
+ *           pointer after the call returns; scratch space comes from the caller
+ *           through (ws, ws_bytes), sized by awq_workspace_bytes().
+ * Layout.   Row-major, innermost index contiguous:
+ *             W       [N][K] fp16      (out_features x in_features; y = X W^T)
+ *             X, Y    [M][K] / [M][N] fp16
+ *             qweight [N][K/8] uint32: the 4-bit code of (n, k) sits in bits
+ *                     4*(k%8) .. 4*(k%8)+3 of word k/8 (little-endian nibbles)
+ *             scales  [N][K/G] fp16
+ *             qzeros  [N][ceil((K/G)/8)] uint32, same nibble order, unused
+ *                     nibbles 0; NULL when zero_point is 0 (implicit zero 8)
+ *           Every pointer must be 16-byte aligned; K must be a multiple of G.
+ * Async.    Calls enqueue work on `stream` and return without synchronising.
+ * Errors.   Argument errors are detected on the host, before anything is
+ *           launched, and return AWQ_ERR_INVALID_ARG / AWQ_ERR_UNSUPPORTED /
+ *           AWQ_ERR_WORKSPACE.  A failed launch returns AWQ_ERR_CUDA.  Device-side
+ *           waits are bounded: a wait that runs out sets a device error word
+ *           and the kernel returns; awq_device_error() reports it as
+ *           AWQ_ERR_TIMEOUT.  NaN or Inf in W or X propagate into the outputs.
+ */
+#ifndef AWQ_B200_H
+#define AWQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* quant_config of the pages: w_bit must be 4, q_group_size one of 32/64/128/256,
+ * zero_point 1 = asymmetric (per-group zero), 0 = symmetric (implicit zero 8). */
+typedef struct awq_quant_config {
+    int32_t w_bit;
+    int32_t q_group_size;
+    int32_t zero_point;
+} awq_quant_config;
+
+typedef enum awq_status {
+    AWQ_OK = 0,
+    AWQ_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size */
+    AWQ_ERR_UNSUPPORTED = 2,   /* valid but not handled (w_bit != 4, group size, M too large for GEMV) */
+    AWQ_ERR_WORKSPACE = 3,     /* ws too small (see awq_workspace_bytes) */
+    AWQ_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed */
+    AWQ_ERR_TIMEOUT = 5        /* a bounded device wait ran out (see awq_device_error) */
+} awq_status;
+
+/* Operation ids for awq_workspace_bytes. */
+enum {
+    AWQ_OP_QUANTIZE_PACK = 0,
+    AWQ_OP_SCALE_SEARCH = 1,
+    AWQ_OP_GEMV = 2,
+    AWQ_OP_GEMM = 3
+};
+
+/* Static string for a status code; never NULL. */
+const char* awq_status_string(awq_status status);
+
+/* ABI version of this header (increases on incompatible change). */
+int32_t awq_abi_version(void);
+
+/*
+ * Group-wise 4-bit quantisation and packing of ws = W * diag(s).
+ * Source: lshu.cn guide, 量化超参数调优 (group size, zero-point); quant_config
+ * block of "Optimization Awq".  Per row n and group g of G input channels, in
+ * IEEE fp32 with round-half-even rint:
+ *   zero_point=1: scale = max((max-min)/15, 1e-5) rounded to fp16 (scale16),
+ *                 zero  = clamp(rint(-min/scale16), 0, 15),
+ *                 q     = clamp(rint(ws/scale16) + zero, 0, 15)
+ *   zero_point=0: scale = max(max|ws|/7, 1e-5) rounded to fp16,
+ *                 q     = clamp(rint(ws/scale16), -8, 7) + 8
+ * ws = fp32(W)*fp32(s) is exact.  s may be NULL (s = 1: plain round-to-nearest).
+ * W [N][K], s [K] -> qweight [N][K/8], scales [N][K/G], qzeros (zero_point=1 only).
+ * Needs no workspace.  N, K > 0.
+ */
+awq_status awq_quantize_pack(const uint16_t* W, const uint16_t* s, int32_t N, int32_t K,
+                             awq_quant_config cfg, uint32_t* qweight, uint16_t* scales,
+                             uint32_t* qzeros, void* stream);
+
+/*
+ * Activation-aware scale search (lshu.cn guide, 算法原理): for alpha_i = i/n_grid,
+ * i = 0 .. n_grid-1, with m_k = mean_t |X[t][k]| (exact, fp64) and
+ * s_i = fp16(max(pow(m_k, alpha_i), 2^-14)), evaluate
+ *   loss_i = mean_{t,n} ( sum_k X[t][k] * (Q(W s_i)/s_i - W)[n][k] )^2
+ * where Q is the group quantiser of awq_quantize_pack with the same cfg, and keep
+ * the smallest (ties to the smaller alpha).  Writes s_out [K] fp16 = s of the
+ * best alpha; losses_out [n_grid] fp64 and best_index_out [1] int32 are DEVICE
+ * pointers and may be NULL.  alpha* = best_index / n_grid.
+ * X [M][K] are the calibration activations (M >= 1 tokens), W [N][K].
+ * 1 <= n_grid <= 64.  ws_bytes >= awq_workspace_bytes(AWQ_OP_SCALE_SEARCH, M, N, K, cfg).
+ * Every fp32 product of the loss uses X exactly and Q(Ws)/s - W split into two
+ * fp16 terms (22-bit significand), accumulated in fp32 on the tensor cores and
+ * summed in fp64.
+ */
+awq_status awq_scale_search(const uint16_t* X, int32_t M, const uint16_t* W, int32_t N,
+                            int32_t K, awq_quant_config cfg, int32_t n_grid, uint16_t* s_out,
+                            double* losses_out, int32_t* best_index_out, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/*
+ * Activation side of the scaling (lshu.cn guide, 算法原理: "s^-1 * X"):
+ * X_out[m][k] = fp16(fp32(X[m][k]) / fp32(s[k])), IEEE division, round to nearest.
+ * The linear entry points take activations already divided this way (in a model
+ * the division folds into the preceding normalisation).  X_out may equal X.
+ */
+awq_status awq_fold_inverse_scale(const uint16_t* X, const uint16_t* s, int32_t M, int32_t K,
+                                  uint16_t* X_out, void* stream);
+
+/*
+ * Fused dequantising linear, single-token / small-batch form ("GEMV", the pages'
+ * WQLinear_GEMV: batch 1 decode).  Y[m][n] = fp16( sum_k X[m][k] *
+ * (q[n][k] - zero[n][k/G]) * scale16[n][k/G] ), products exact, fp32 accumulation.
+ * 1 <= M <= 8 (memory-bound for M <= 2; larger batches belong to awq_linear_gemm).
+ * Needs no workspace (ws may be NULL).
+ */
+awq_status awq_linear_gemv(const uint16_t* X, int32_t M, const uint32_t* qweight,
+                           const uint16_t* scales, const uint32_t* qzeros, int32_t N, int32_t K,
+                           awq_quant_config cfg, uint16_t* Y, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/*
+ * Fused dequantising linear, batched / prefill form ("GEMM", the pages'
+ * WQLinear_GEMM, the default for batch > 1).  Same result definition as
+ * awq_linear_gemv; the weight tile is dequantised to fp16 ((q-zero)*scale16,
+ * one rounding) in shared memory and multiplied on the tcgen05 tensor cores with
+ * fp32 accumulation in tensor memory.  Any M >= 1.  Needs no workspace.
+ */
+awq_status awq_linear_gemm(const uint16_t* X, int32_t M, const uint32_t* qweight,
+                           const uint16_t* scales, const uint32_t* qzeros, int32_t N, int32_t K,
+                           awq_quant_config cfg, uint16_t* Y, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Workspace bytes an operation needs for the given sizes (0 = none). */
+size_t awq_workspace_bytes(int32_t op, int32_t M, int32_t N, int32_t K, awq_quant_config cfg);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device: AWQ_ERR_TIMEOUT if a bounded device wait ran out since the
+ * last call, AWQ_ERR_CUDA if the synchronisation itself failed, else AWQ_OK.
+ */
+awq_status awq_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_B200_H */

@@ -18,5 +18,7 @@ def lib():
     import torch
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    from bit_weight_only_linear_b200 import awq
+    from bit_weight_only_linear_b200 import awq, build
+    build.build()
+    awq.load_library()
     return awq

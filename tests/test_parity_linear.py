@@ -1,0 +1,80 @@
+"""GPU parity: awq_linear_gemv / awq_linear_gemm against the oracle's fp64 linear.
+
+Tolerance (from the arithmetic): |y - y_ref| <= 1e-2 (|y_ref| + rms(y_ref)) per element.
+The kernels' own error is far smaller (exact fp16 products, fp32 accumulation, one fp16
+rounding of the output; the GEMM adds one fp16 rounding of each dequantised weight)."""
+import numpy as np
+import pytest
+import torch
+
+import inputs
+from helpers import assert_linear_close, to_dev, to_np
+from oracle import awq_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _packed(W, G, zp, s=None):
+    q, sc, z = O.quantize_pack(W, s, G, zp)
+    return q, sc, z, (to_dev(q), to_dev(sc), to_dev(z) if zp else None)
+
+
+def _run(lib, kind, X, dq, G, zp):
+    fn = lib.linear_gemv if kind == "gemv" else lib.linear_gemm
+    y = fn(to_dev(X), dq[0], dq[1], dq[2], G, zp)
+    torch.cuda.synchronize()
+    return to_np(y)
+
+
+SMALL = [(1, 128, 8), (1, 256, 37), (2, 1024, 64), (3, 2048, 130), (4, 4096, 96), (8, 3072, 33),
+         (1, 4096 + 1024, 257), (5, 256, 512), (1, 14336, 64)]
+
+
+@pytest.mark.parametrize("G", O.GROUP_SIZES)
+@pytest.mark.parametrize("zp", [True, False])
+@pytest.mark.parametrize("mkn", SMALL, ids=lambda t: "x".join(map(str, t)))
+def test_gemv_parity(lib, G, zp, mkn):
+    M, K, N = mkn
+    if K % G:
+        pytest.skip("K % G")
+    W = inputs.weights(N, K, 0.02, seed=200 + K + N)
+    X = inputs.activations(M, K, seed=201 + M + K)
+    q, sc, z, dq = _packed(W, G, zp)
+    y = _run(lib, "gemv", X, dq, G, zp)
+    assert_linear_close(y, O.linear(X, q, sc, z, K, G, zp))
+
+
+def test_gemv_outputs_do_not_spill(lib):
+    """Guard band around Y: the kernel writes exactly M x N values."""
+    M, K, N, G = 3, 1024, 70, 64
+    W = inputs.weights(N, K, seed=202)
+    X = inputs.activations(M, K, seed=203)
+    q, sc, z, dq = _packed(W, G, True)
+    buf = torch.full((M * N + 64,), float("nan"), dtype=torch.float16, device="cuda")
+    y = buf[32:32 + M * N].view(M, N)
+    lib.linear_gemv(to_dev(X), dq[0], dq[1], dq[2], G, True, out=y)
+    torch.cuda.synchronize()
+    b = to_np(buf).astype(np.float64)
+    assert np.all(np.isnan(b[:32])) and np.all(np.isnan(b[32 + M * N:]))
+    assert_linear_close(b[32:32 + M * N].reshape(M, N), O.linear(X, q, sc, z, K, G, True))
+
+
+def test_gemv_single_workload_full(lib):
+    """M=1, K=N=4096, G=128, zero point: every output against the oracle."""
+    W = inputs.weights(4096, 4096, 0.02, seed=inputs.SEED_W)
+    X = inputs.activations(1, 4096, seed=inputs.SEED_X)
+    q, sc, z, dq = _packed(W, 128, True)
+    assert_linear_close(_run(lib, "gemv", X, dq, 128, True), O.linear(X, q, sc, z, 4096, 128, True))
+
+
+def test_gemv_mistral_layer_sampled(lib):
+    """The seven Mistral-7B decode linears at M=1 (full size, launch as benchmarked):
+    256 sampled output channels per linear against the oracle."""
+    rng = np.random.Generator(np.random.PCG64(5))
+    for name, W, X in inputs.layer_inputs(inputs.MISTRAL_7B_LAYER, 1, 0.02):
+        N, K = W.shape
+        q, sc, z, dq = _packed(W, 128, True)
+        y = _run(lib, "gemv", X, dq, 128, True)
+        rows = np.sort(rng.choice(N, 256, replace=False))
+        ref = O.linear_rows(X, q, sc, z, K, 128, True, rows)
+        assert_linear_close(y[:, rows], ref)
