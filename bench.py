@@ -227,24 +227,34 @@ def time_decode(awq, torch, layers, steps, warmup, world):
     return ms, steps
 
 
-def per_launch_gemv(awq, torch, layers, reps=50):
-    """Average duration of each GEMV launch (CUDA events on the launching stream), for
-    the roofline object."""
+def per_launch_gemv(awq, torch, layers, reps=64):
+    """Average device duration of each GEMV launch, for the roofline object: a CUDA
+    graph of `reps` launches of one linear (rotating weight copies), timed with CUDA
+    events on the stream it is replayed on."""
     out = []
-    s = torch.cuda.current_stream()
+    stream = torch.cuda.Stream()
     for L in layers:
-        for r in range(ROTATIONS):
-            q, sc, z = L["copies"][r]
-            awq.linear_gemv(L["x"], q, sc, z, G, ZP, out=L["y"])
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for r in range(ROTATIONS):
+                q, sc, z = L["copies"][r]
+                awq.linear_gemv(L["x"], q, sc, z, G, ZP, out=L["y"])
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(reps):
+                q, sc, z = L["copies"][i % ROTATIONS]
+                awq.linear_gemv(L["x"], q, sc, z, G, ZP, out=L["y"])
+        g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(s)
-        for i in range(reps):
-            q, sc, z = L["copies"][i % ROTATIONS]
-            awq.linear_gemv(L["x"], q, sc, z, G, ZP, out=L["y"])
-        e1.record(s)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(3):
+                g.replay()
+            e1.record(stream)
         torch.cuda.synchronize()
-        out.append((L["name"], linear_bytes(1, L["N"], L["K"]), e0.elapsed_time(e1) / reps))
+        out.append((L["name"], linear_bytes(1, L["N"], L["K"]), e0.elapsed_time(e1) / (3 * reps)))
+        del g
     return out
 
 

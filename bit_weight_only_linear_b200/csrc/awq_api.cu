@@ -81,26 +81,40 @@ awq_status check_linear(const uint16_t* X, int M, const uint32_t* qweight, const
     return AWQ_OK;
 }
 
-template <int MT>
+template <int WT>
 awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
                        const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
                        cudaStream_t st) {
-    constexpr int R = gemv_rows_per_warp(MT);
     DeviceInfo d;
     if (!device_info(d)) return AWQ_ERR_CUDA;
-    const size_t smem = gemv_smem_bytes(MT, K);
+    const int nsteps = K / (32 * WT);
+    const size_t smem = GemvSmem::bytes(M, K, nsteps);
     if (smem > (size_t)d.max_smem_optin) return AWQ_ERR_UNSUPPORTED;
-    auto kern = gemv_kernel<MT, R>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    auto kern = gemv_mma_kernel<WT>;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return AWQ_ERR_CUDA;
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvThreads, smem) != cudaSuccess || occ < 1)
         return AWQ_ERR_CUDA;
-    const int row_groups = ceil_div(N, R);
-    const int want = ceil_div(row_groups, kGemvWarps);
-    const int grid = want < d.sms * occ ? want : d.sms * occ;
-    kern<<<grid, kGemvThreads, smem, st>>>(X, M, qweight, scales, qzeros, N, K, cfg.q_group_size,
-                                           cfg.zero_point, Y);
+    // persistent grid: at most one wave, row groups spread evenly over the CTAs
+    const int n_rg = ceil_div(N, kGemvRows);
+    const int slots = d.sms * occ;
+    const int per_cta = ceil_div(n_rg, slots);
+    const int grid = ceil_div(n_rg, per_cta);
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(grid);
+    lc.blockDim = dim3(kGemvThreads);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&lc, kern, X, M, qweight, scales, qzeros, N, K, (int)cfg.q_group_size,
+                           (int)cfg.zero_point, Y) != cudaSuccess)
+        return AWQ_ERR_CUDA;
     return launch_status();
 }
 
@@ -158,12 +172,13 @@ awq_status awq_linear_gemv(const uint16_t* X, int32_t M, const uint32_t* qweight
     (void)ws_bytes;
     awq_status st = check_linear(X, M, qweight, scales, qzeros, N, K, cfg, Y);
     if (st != AWQ_OK) return st;
+    if (M > 8) return AWQ_ERR_UNSUPPORTED;
     cudaStream_t s = (cudaStream_t)stream;
-    if (M == 1) return launch_gemv<1>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-    if (M == 2) return launch_gemv<2>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-    if (M <= 4) return launch_gemv<4>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-    if (M <= 8) return launch_gemv<8>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-    return AWQ_ERR_UNSUPPORTED;
+    switch (cfg.q_group_size) {
+        case 32: return launch_gemv<1>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+        case 64: return launch_gemv<2>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+        default: return launch_gemv<4>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+    }
 }
 
 awq_status awq_linear_gemm(const uint16_t* X, int32_t M, const uint32_t* qweight, const uint16_t* scales,

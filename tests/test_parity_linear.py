@@ -78,3 +78,75 @@ def test_gemv_mistral_layer_sampled(lib):
         rows = np.sort(rng.choice(N, 256, replace=False))
         ref = O.linear_rows(X, q, sc, z, K, 128, True, rows)
         assert_linear_close(y[:, rows], ref)
+
+
+GEMM_SMALL = [(1, 128, 128), (4, 256, 130), (16, 1024, 256), (17, 512, 384), (33, 256, 128),
+              (64, 2048, 256), (100, 1024, 200), (128, 512, 128), (200, 256, 384), (256, 1024, 256),
+              (300, 512, 136), (513, 256, 128)]
+
+
+@pytest.mark.parametrize("G", O.GROUP_SIZES)
+@pytest.mark.parametrize("zp", [True, False])
+@pytest.mark.parametrize("mkn", GEMM_SMALL, ids=lambda t: "x".join(map(str, t)))
+def test_gemm_parity(lib, G, zp, mkn):
+    M, K, N = mkn
+    if K % G:
+        pytest.skip("K % G")
+    W = inputs.weights(N, K, 0.02, seed=300 + K + N)
+    X = inputs.activations(M, K, seed=301 + M + K)
+    q, sc, z, dq = _packed(W, G, zp)
+    y = _run(lib, "gemm", X, dq, G, zp)
+    assert_linear_close(y, O.linear(X, q, sc, z, K, G, zp))
+
+
+def test_gemm_ragged_k_tail(lib):
+    """K = 96 with G = 32: the last 64-channel k-block is half outside the matrix."""
+    M, K, N, G = 40, 96, 130, 32
+    W = inputs.weights(N, K, seed=302)
+    X = inputs.activations(M, K, seed=303)
+    for zp in (True, False):
+        q, sc, z, dq = _packed(W, G, zp)
+        assert_linear_close(_run(lib, "gemm", X, dq, G, zp), O.linear(X, q, sc, z, K, G, zp))
+
+
+def test_gemm_outputs_do_not_spill(lib):
+    M, K, N, G = 70, 512, 136, 128
+    W = inputs.weights(N, K, seed=304)
+    X = inputs.activations(M, K, seed=305)
+    q, sc, z, dq = _packed(W, G, True)
+    buf = torch.full((M * N + 64,), float("nan"), dtype=torch.float16, device="cuda")
+    y = buf[32:32 + M * N].view(M, N)
+    lib.linear_gemm(to_dev(X), dq[0], dq[1], dq[2], G, True, out=y)
+    torch.cuda.synchronize()
+    lib.device_error()
+    b = to_np(buf).astype(np.float64)
+    assert np.all(np.isnan(b[:32])) and np.all(np.isnan(b[32 + M * N:]))
+    assert_linear_close(b[32:32 + M * N].reshape(M, N), O.linear(X, q, sc, z, K, G, True))
+
+
+def test_gemm_equals_gemv_at_small_batch(lib):
+    """Both forms compute the same definition: at M = 4 they agree within the rule."""
+    M, K, N, G = 4, 4096, 1024, 128
+    W = inputs.weights(N, K, seed=306)
+    X = inputs.activations(M, K, seed=307)
+    q, sc, z, dq = _packed(W, G, True)
+    a = _run(lib, "gemv", X, dq, G, True)
+    b = _run(lib, "gemm", X, dq, G, True)
+    assert_linear_close(b, a.astype(np.float64))
+
+
+def test_gemm_llama70b_prefill_sampled(lib):
+    """The four Llama-70B-shaped prefill linears at M = 2048, full size, launched as
+    benchmarked: 128 sampled output channels each against the oracle."""
+    rng = np.random.Generator(np.random.PCG64(9))
+    for i, (name, K, N) in enumerate(inputs.LLAMA_70B_FUSED):
+        W = inputs.weights(N, K, 0.015, inputs.SEED_W + 30 + i)
+        X = inputs.activations(2048, K, inputs.SEED_X + 30 + i, inputs.SEED_OUTLIER + 30)
+        Wd = to_dev(W)
+        q, sc, z = lib.quantize_pack(Wd, None, 128, True)
+        del Wd
+        y = to_np(lib.linear_gemm(to_dev(X), q, sc, z, 128, True))
+        lib.device_error()
+        rows = np.sort(rng.choice(N, 128, replace=False))
+        ref = O.linear_rows(X, to_np(q), to_np(sc), to_np(z), K, 128, True, rows)
+        assert_linear_close(y[:, rows], ref)
