@@ -81,7 +81,7 @@ awq_status check_linear(const uint16_t* X, int M, const uint32_t* qweight, const
     return AWQ_OK;
 }
 
-template <int WT>
+template <int WT, bool ONE>
 awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
                        const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
                        cudaStream_t st) {
@@ -90,18 +90,22 @@ awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const 
     const int nsteps = K / (32 * WT);
     const size_t smem = GemvSmem::bytes(M, K, nsteps);
     if (smem > (size_t)d.max_smem_optin) return AWQ_ERR_UNSUPPORTED;
-    auto kern = gemv_mma_kernel<WT>;
+    auto kern = gemv_mma_kernel<WT, ONE>;
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return AWQ_ERR_CUDA;
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvThreads, smem) != cudaSuccess || occ < 1)
         return AWQ_ERR_CUDA;
-    // persistent grid: at most one wave, row groups spread evenly over the CTAs
-    const int n_rg = ceil_div(N, kGemvRows);
+    // persistent grid: at most one wave, row-group iterations spread evenly over the CTAs
+    constexpr int UK = kGemvUnitWords / WT;
+    const int units = ceil_div(nsteps, UK);
     const int slots = d.sms * occ;
-    const int per_cta = ceil_div(n_rg, slots);
-    const int grid = ceil_div(n_rg, per_cta);
+    const int ks = gemv_ks(units, ceil_div(N, kGemvRows), slots);
+    const int rpi = kGemvWarps / ks;
+    const int n_it = ceil_div(ceil_div(N, kGemvRows), rpi);
+    const int per_cta = ceil_div(n_it, slots);
+    const int grid = ceil_div(n_it, per_cta);
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(grid);
     lc.blockDim = dim3(kGemvThreads);
@@ -113,9 +117,73 @@ awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const 
     lc.attrs = attr;
     lc.numAttrs = 1;
     if (cudaLaunchKernelEx(&lc, kern, X, M, qweight, scales, qzeros, N, K, (int)cfg.q_group_size,
+                           (int)cfg.zero_point, ks, Y) != cudaSuccess)
+        return AWQ_ERR_CUDA;
+    return launch_status();
+}
+
+template <int WT, bool ONE>
+awq_status launch_gemv_tma(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
+                           const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
+                           cudaStream_t st) {
+    DeviceInfo d;
+    if (!device_info(d)) return AWQ_ERR_CUDA;
+    const GemvTmaSmem L(M, K, cfg.q_group_size);
+    const size_t smem = L.bytes();
+    // qweight [N][K/8] words viewed as {16 words, N rows, K/128 blocks}
+    CUtensorMap tq;
+    if (!make_tmap_3d(&tq, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 16, (uint64_t)N, (uint64_t)(K / 128),
+                      (uint64_t)K / 2, 64, 16, kGemvRows, kTmaKC / 128))
+        return AWQ_ERR_CUDA;
+    if (smem > (size_t)d.max_smem_optin) return AWQ_ERR_UNSUPPORTED;
+    auto kern = gemv_tma_kernel<WT, ONE>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return AWQ_ERR_CUDA;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kTmaThreads, smem) != cudaSuccess || occ < 1)
+        return AWQ_ERR_CUDA;
+    const int n_rg = N / kGemvRows;
+    const int slots = d.sms * occ;
+    const int per_cta = ceil_div(n_rg, slots);
+    const int grid = ceil_div(n_rg, per_cta);
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(grid);
+    lc.blockDim = dim3(kTmaThreads);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&lc, kern, tq, X, M, scales, qzeros, N, K, (int)cfg.q_group_size,
                            (int)cfg.zero_point, Y) != cudaSuccess)
         return AWQ_ERR_CUDA;
     return launch_status();
+}
+
+template <bool ONE>
+awq_status dispatch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
+                         const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
+                         cudaStream_t s) {
+    // every row group full, K in whole 128-code blocks, parameters 16-byte aligned and
+    // the staging fits: TMA path
+    DeviceInfo d;
+    if (!device_info(d)) return AWQ_ERR_CUDA;
+    if (N % kGemvRows == 0 && K % 128 == 0 && (uintptr_t)scales % 16 == 0 &&
+        (!cfg.zero_point || (uintptr_t)qzeros % 16 == 0) &&
+        GemvTmaSmem(M, K, cfg.q_group_size).bytes() <= (size_t)d.max_smem_optin) {
+        switch (cfg.q_group_size) {
+            case 32: return launch_gemv_tma<1, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+            case 64: return launch_gemv_tma<2, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+            default: return launch_gemv_tma<4, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+        }
+    }
+    switch (cfg.q_group_size) {
+        case 32: return launch_gemv<1, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+        case 64: return launch_gemv<2, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+        default: return launch_gemv<4, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+    }
 }
 
 }  // namespace
@@ -174,11 +242,8 @@ awq_status awq_linear_gemv(const uint16_t* X, int32_t M, const uint32_t* qweight
     if (st != AWQ_OK) return st;
     if (M > 8) return AWQ_ERR_UNSUPPORTED;
     cudaStream_t s = (cudaStream_t)stream;
-    switch (cfg.q_group_size) {
-        case 32: return launch_gemv<1>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-        case 64: return launch_gemv<2>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-        default: return launch_gemv<4>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-    }
+    return M == 1 ? dispatch_gemv<true>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s)
+                  : dispatch_gemv<false>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
 }
 
 awq_status awq_linear_gemm(const uint16_t* X, int32_t M, const uint32_t* qweight, const uint16_t* scales,

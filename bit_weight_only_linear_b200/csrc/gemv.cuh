@@ -8,10 +8,10 @@
 // Why this shape (measured on B200): at M = 1 the kernel must turn 0.5 B of codes
 // into one multiply-add at ~12.8 T codes/s to keep up with HBM.  On the CUDA cores
 // the cheapest exact form (mask + fma.rn.f32.f16) costs ~2 issue slots per code and
-// the mixed-precision FMA runs at 19 T/s, so the multiply-adds would saturate the
-// SM.  Here each code costs ~0.7 integer instructions, and the multiply-adds go to
-// the tensor cores through mma.sync m16n8k16 straight from registers (no shared
-// memory round trip), which also makes M = 2..8 free: the MMA's n8 side is the batch.
+// the mixed-precision FMA runs at 19 T/s, so the multiply-adds would saturate the SM.
+// Here each code costs ~0.6 integer instructions, and the multiply-adds go to the
+// tensor cores through mma.sync m16n8k16 straight from registers (no shared-memory
+// round trip), which also makes M = 2..8 free: the MMA's n8 side is the batch.
 //
 //   * Codes become fp16 with a single AND: masking a word with 0x000F000F leaves two
 //     fp16 SUBNORMALS q * 2^-24 (codes 0 and 4 of the word), 0x00F000F0 leaves
@@ -21,44 +21,62 @@
 //   * The k order inside an MMA is free as long as A and B agree: lane (g, t) feeds
 //     the k-slots of its quad with codes of its own word, and X is staged in shared
 //     memory permuted the same way, so no shuffles or byte permutes are needed.
-//   * The 4 lanes of a quad cover 32*WT consecutive codes (WT = 1, 2, 4 words each
-//     for G = 32, 64, >= 128), which always lie inside one group, so after each
-//     k-step the group's scale and zero point are applied once in fp32:
-//       y += scale16 * (2^24 (D1 + D16/16) - z * sum_k x).
-//   * Persistent CTAs: each stages X once and then walks row groups of 16 output
-//     channels (rg = blockIdx.x, blockIdx.x + gridDim.x, ...).  Its 8 warps split K;
-//     each warp keeps kGemvDepth k-steps of loads in flight across row-group
-//     boundaries (a ring in registers), so the next row group streams in while the
-//     current one is multiplied.  Per row group the 8 partial sums are added in a
-//     fixed order (deterministic) through a double-buffered shared-memory slot.
+//   * The 4 lanes of a quad cover one k-step of 32*WT consecutive codes (WT = 1, 2, 4
+//     words each for G = 32, 64, >= 128), which always lies inside one group, so after
+//     each k-step the group's scale and zero point are applied once in fp32:
+//       y += (scale16 * 2^24) (D1 + D16/16) - (scale16 * z) sum_k x.
+//   * A unit is UK k-steps (8 words per row per lane).  Loads are never predicated:
+//     rows past N are read from row N-1 and dropped at the store, k-steps past the
+//     end are read from the last one with their scale forced to 0.
+//   * Persistent CTAs stage X once, then walk row-group iterations.  KS warps split
+//     the K of one 16-row group (KS = 1..8, chosen so that each warp has >= 4 units);
+//     the CTA's 8 warps work on 8/KS row groups at a time.  Each warp keeps kGemvDepth
+//     units of loads in flight across iterations (a ring in registers; loaded values
+//     are stored untouched, since using a value stalls on its load).  Per iteration
+//     the KS partial sums of a row are added in a fixed order (deterministic).
 //   * Programmatic dependent launch: weight loads are issued before
 //     griddepcontrol.wait, so they overlap the previous kernel's tail; only X (the
 //     previous layer's output in a model) is read after it.
 #pragma once
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace awq {
 
 constexpr int kGemvThreads = 256;
 constexpr int kGemvWarps = 8;
-constexpr int kGemvRows = 16;      // output channels per CTA (MMA M)
-constexpr int kGemvDepth = 4;      // k-steps of loads in flight per warp
+constexpr int kGemvRows = 16;      // output channels per row group (MMA M)
+constexpr int kGemvDepth = 2;      // units of loads in flight per warp
+constexpr int kGemvUnitWords = 8;  // code words per row per lane per unit
 
 __host__ __device__ constexpr int gemv_words_per_thread(int G) { return G >= 128 ? 4 : G / 32; }
 
 struct GemvSmem {
     // X permuted: [m][kstep][j][t] uint4, row pitch padded by 64 B; then xsum [m][kstep] fp32;
-    // then partials [2 slots][warp][16 rows][8 m] fp32.
+    // then partials [2 slots][8 warps][16 rows][8 m] fp32; then a 64-byte zero row.
     static __host__ __device__ inline size_t x_pitch(int K) { return (size_t)K * 2 + 64; }
     static __host__ __device__ inline size_t xsum_off(int M, int K) { return (size_t)M * x_pitch(K); }
     static __host__ __device__ inline size_t part_off(int M, int K, int nsteps) {
         return (xsum_off(M, K) + (size_t)M * nsteps * 4 + 15) & ~(size_t)15;
     }
-    static __host__ __device__ inline size_t bytes(int M, int K, int nsteps) {
+    static __host__ __device__ inline size_t zero_off(int M, int K, int nsteps) {
         return part_off(M, K, nsteps) + (size_t)2 * kGemvWarps * kGemvRows * 8 * 4;
     }
+    static __host__ __device__ inline size_t bytes(int M, int K, int nsteps) { return zero_off(M, K, nsteps) + 64; }
 };
+
+// K-split of one row group over KS warps: split further while a warp keeps at
+// least 4 units, or (small N) while there are fewer row-group iterations than
+// resident CTAs and a warp keeps at least one unit.
+__host__ __device__ inline int gemv_ks(int units_per_row_group, int row_groups, int slots) {
+    int ks = 1;
+    while (ks < kGemvWarps &&
+           (units_per_row_group >= 8 * ks ||
+            (units_per_row_group >= 2 * ks && row_groups * ks / kGemvWarps < slots)))
+        ks <<= 1;
+    return ks;
+}
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -69,39 +87,49 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One k-step of loads in flight.  Everything is kept exactly as loaded: using a
-// loaded value (even to pack or shift it) would stall the thread on the load.
-template <int WT>
-struct GemvStep {
-    uint32_t wa[WT], wb[WT];   // code words of rows g and g+8
-    uint32_t sa, sb;           // scale16 bits of rows g and g+8
-    uint32_t za, zb;           // packed zero words of rows g and g+8
-};
-
-template <int WT>
-__device__ __forceinline__ void load_words(const uint32_t* p, uint32_t (&w)[WT]) {
-    if constexpr (WT == 4) {
-        uint4 v;
-        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                     : "l"(p));
-        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-    } else if constexpr (WT == 2) {
-        uint2 v;
-        asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-        w[0] = v.x; w[1] = v.y;
-    } else {
-        asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(w[0]) : "l"(p));
-    }
+// D = A * B (accumulator starts from zero).
+__device__ __forceinline__ void mma_16816_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                uint32_t b0, uint32_t b1) {
+    const float z = 0.0f;
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
 }
 
 template <int WT>
+__device__ __forceinline__ void load_words(const uint32_t* p, uint32_t* w) {
+    if constexpr (WT == 4) {
+        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "l"(p));
+    } else if constexpr (WT == 2) {
+        asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "l"(p));
+    } else {
+        asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(w[0]) : "l"(p));
+    }
+}
+
+// One unit of loads in flight (UK k-steps of rows g and g+8), kept exactly as loaded.
+// A unit covers 256 consecutive codes starting at a multiple of 256, i.e. 256/G whole
+// groups (or part of one when G = 256) starting at a multiple of 256/G, so all of
+// its zero points sit in one packed zero word (8 groups per word).
+template <int UK>
+struct GemvUnit {
+    uint32_t wa[kGemvUnitWords], wb[kGemvUnitWords];   // code words of rows g and g+8
+    uint32_t sa[UK], sb[UK];                           // scale16 bits per k-step
+    uint32_t za, zb;                                   // packed zero word of the unit
+};
+
+template <int WT, bool ONE>
 __global__ void __launch_bounds__(kGemvThreads, 2)
 gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restrict__ qweight,
                 const uint16_t* __restrict__ scales, const uint32_t* __restrict__ qzeros, int N, int K, int G,
-                int zero_point, uint16_t* __restrict__ Y) {
-    extern __shared__ __align__(16) uint8_t smem[];
+                int zero_point, int ks_arg, uint16_t* __restrict__ Y) {
+    constexpr int UK = kGemvUnitWords / WT;   // k-steps per unit
     constexpr int kStepCodes = 32 * WT;
+    extern __shared__ __align__(16) uint8_t smem[];
     const int nsteps = K / kStepCodes;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -111,57 +139,56 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
     const int ng = K / G;
     const int nzw = (ng + 7) >> 3;
     const bool zp = zero_point != 0;
-
-    // The units of this warp are (row group, k-step) pairs: row groups
-    // blockIdx.x + r * gridDim.x (r = 0 .. my_rg-1), k-steps s_begin .. s_begin+per-1 of
-    // each.  k-steps at or beyond nsteps are empty, so every warp has the same unit
-    // count and the per-row-group barrier below is uniform.  Cursors advance by one
-    // unit at a time (no divisions in the loop).
-    const int per = (nsteps + kGemvWarps - 1) / kGemvWarps;
-    const int s_begin = warp * per;
-    const int n_rg = (N + kGemvRows - 1) / kGemvRows;
-    const int my_rg = blockIdx.x < n_rg ? (n_rg - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int U = my_rg * per;
     const int lg = 31 - __clz(G);            // G is a power of two
 
-    // load cursor
-    int l_rg = blockIdx.x, l_i = 0;
-    auto load_next = [&](GemvStep<WT>& st) {
-        const int s = s_begin + l_i;
-        const int ra = l_rg * kGemvRows + g;
-        const bool va = ra < N && s < nsteps, vb = ra + 8 < N && s < nsteps;
-        const uint32_t* qa = qweight + (size_t)ra * kw + (s * 4 * WT + t * WT);
-        const int grp = (s * kStepCodes) >> lg;
-        if (va) {
-            load_words<WT>(qa, st.wa);
-        } else {
+    // K split: KS warps per row group, RPI = 8/KS row groups per CTA iteration.
+    const int units = (nsteps + UK - 1) / UK;                 // units per row group
+    const int KS = ks_arg;
+    const int RPI = kGemvWarps / KS;
+    const int sub = warp / KS;                                // which row group of the iteration
+    const int kpart = warp - sub * KS;                        // which K part
+    const int per = (units + KS - 1) / KS;                    // units per warp per row group
+    const int u_begin = kpart * per;
+    const int n_rg = (N + kGemvRows - 1) / kGemvRows;
+    const int n_it = (n_rg + RPI - 1) / RPI;                  // row-group iterations in total
+    const int my_it = blockIdx.x < n_it ? (n_it - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int U = my_it * per;                                // units of this warp
+
+    // load cursor: iteration l_it (row group l_it * RPI + sub), unit u_begin + l_i
+    int l_it = blockIdx.x, l_i = 0;
+    auto load_next = [&](GemvUnit<UK>& st) {
+        const int rg = l_it * RPI + sub;
+        const int ra = min(rg * kGemvRows + g, N - 1);
+        const int rb = min(rg * kGemvRows + g + 8, N - 1);
+        const uint32_t* qa = qweight + (size_t)ra * kw + t * WT;
+        const uint32_t* qb = qweight + (size_t)rb * kw + t * WT;
+        const int s0 = (u_begin + l_i) * UK;
+        const uint16_t* spa = scales + (size_t)ra * ng;
+        const uint16_t* spb = scales + (size_t)rb * ng;
 #pragma unroll
-            for (int j = 0; j < WT; ++j) st.wa[j] = 0;
+        for (int k = 0; k < UK; ++k) {
+            const int s = min(s0 + k, nsteps - 1);
+            load_words<WT>(qa + s * 4 * WT, st.wa + k * WT);
+            load_words<WT>(qb + s * 4 * WT, st.wb + k * WT);
+            const int grp = (s * kStepCodes) >> lg;
+            st.sa[k] = __ldg(spa + grp);
+            st.sb[k] = __ldg(spb + grp);
         }
-        if (vb) {
-            load_words<WT>(qa + 8 * (size_t)kw, st.wb);
-        } else {
-#pragma unroll
-            for (int j = 0; j < WT; ++j) st.wb[j] = 0;
-        }
-        const uint16_t* sp = scales + (size_t)ra * ng + grp;
-        st.sa = va ? __ldg(sp) : 0u;
-        st.sb = vb ? __ldg(sp + 8 * (size_t)ng) : 0u;
         if (zp) {
-            const uint32_t* zpp = qzeros + (size_t)ra * nzw + (grp >> 3);
-            st.za = va ? __ldg(zpp) : 0u;
-            st.zb = vb ? __ldg(zpp + 8 * (size_t)nzw) : 0u;
+            const int grp0 = (min(s0, nsteps - 1) * kStepCodes) >> lg;
+            st.za = __ldg(qzeros + (size_t)ra * nzw + (grp0 >> 3));
+            st.zb = __ldg(qzeros + (size_t)rb * nzw + (grp0 >> 3));
         } else {
             st.za = st.zb = 0x88888888u;   // implicit zero 8 in every nibble
         }
         if (++l_i == per) {
             l_i = 0;
-            l_rg += gridDim.x;
+            l_it += gridDim.x;
         }
     };
 
     // 1. weights first (they do not depend on the previous kernel)
-    GemvStep<WT> buf[kGemvDepth];
+    GemvUnit<UK> buf[kGemvDepth];
 #pragma unroll
     for (int i = 0; i < kGemvDepth; ++i)
         if (i < U) load_next(buf[i]);
@@ -202,6 +229,8 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
             }
         }
     }
+    if (threadIdx.x < 16)
+        reinterpret_cast<uint32_t*>(smem + GemvSmem::zero_off(M, K, nsteps))[threadIdx.x] = 0u;
     __syncthreads();
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // per-(m, k-step) sums of x, from shared memory, in a fixed order
@@ -223,47 +252,63 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
 
     // 3. stream the units; D fragment: y[0] = (row g, col 2t), y[1] = (g, 2t+1),
     //    y[2] = (g+8, 2t), y[3] = (g+8, 2t+1)
-    const bool bm = g < M;   // lane supplies B column g
-    const uint8_t* xrow = smem + g * pitch + t * 16;
+    // lanes whose B column is past M read the zero row staged after X
+    const uint8_t* xrow = (g < M ? smem + g * pitch : smem + GemvSmem::zero_off(M, K, nsteps)) + t * 16;
+    const size_t xstep = g < M ? 64 : 0;
     const int m0 = 2 * t, m1 = 2 * t + 1;
-    const float* xs0 = xsum + m0 * nsteps;
-    const float* xs1 = xsum + m1 * nsteps;
+    const float* xs0 = xsum + (m0 < M ? m0 : 0) * nsteps;
+    const float* xs1 = xsum + (m1 < M ? m1 : 0) * nsteps;
+    const float xm0 = m0 < M ? 1.0f : 0.0f, xm1 = m1 < M ? 1.0f : 0.0f;
     float y[4] = {0.f, 0.f, 0.f, 0.f};
-    int c_rg = blockIdx.x, c_i = 0, c_r = 0;   // consume cursor
+    int c_it = blockIdx.x, c_i = 0, c_r = 0;   // consume cursor
     for (int u0 = 0; u0 < U; u0 += kGemvDepth) {
 #pragma unroll
         for (int i = 0; i < kGemvDepth; ++i) {
             if (u0 + i >= U) break;
-            const int s = s_begin + c_i;
-            if (s < nsteps) {
-                GemvStep<WT>& st = buf[i];
-                float d1[4] = {0.f, 0.f, 0.f, 0.f}, d16[4] = {0.f, 0.f, 0.f, 0.f};
+            GemvUnit<UK>& st = buf[i];
+            const int s0 = (u_begin + c_i) * UK;
+#pragma unroll
+            for (int k = 0; k < UK; ++k) {
+                const int s = s0 + k;
+                const int sc = min(s, nsteps - 1);
+                float d1[4], d16[4];
 #pragma unroll
                 for (int j = 0; j < WT; ++j) {
-                    uint4 b = make_uint4(0, 0, 0, 0);
-                    if (bm) b = *reinterpret_cast<const uint4*>(xrow + (size_t)(s * WT + j) * 64);
-                    const uint32_t wa = st.wa[j], wb = st.wb[j];
+                    const uint4 b = *reinterpret_cast<const uint4*>(xrow + (size_t)(sc * WT + j) * xstep);
+                    const uint32_t wa = st.wa[k * WT + j], wb = st.wb[k * WT + j];
                     const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
-                    mma_16816(d1, wa & 0x000F000Fu, wb & 0x000F000Fu, wa8 & 0x000F000Fu, wb8 & 0x000F000Fu, b.x, b.y);
-                    mma_16816(d16, wa & 0x00F000F0u, wb & 0x00F000F0u, wa8 & 0x00F000F0u, wb8 & 0x00F000F0u, b.z,
-                              b.w);
+                    if (j == 0) {
+                        mma_16816_first(d1, wa & 0x000F000Fu, wb & 0x000F000Fu, wa8 & 0x000F000Fu,
+                                        wb8 & 0x000F000Fu, b.x, b.y);
+                        mma_16816_first(d16, wa & 0x00F000F0u, wb & 0x00F000F0u, wa8 & 0x00F000F0u,
+                                        wb8 & 0x00F000F0u, b.z, b.w);
+                    } else {
+                        mma_16816(d1, wa & 0x000F000Fu, wb & 0x000F000Fu, wa8 & 0x000F000Fu, wb8 & 0x000F000Fu,
+                                  b.x, b.y);
+                        mma_16816(d16, wa & 0x00F000F0u, wb & 0x00F000F0u, wa8 & 0x00F000F0u, wb8 & 0x00F000F0u,
+                                  b.z, b.w);
+                    }
                 }
-                // fold this k-step's group scale and zero point (fp32); the 4-bit zero
-                // becomes a float through the 2^23 magic number
-                const float sa = h2f((uint16_t)st.sa), sb = h2f((uint16_t)st.sb);
-                const int zsh = 4 * (((s * kStepCodes) >> lg) & 7);
+                // fold the k-step's group scale and zero point; k-steps past the end get scale 0
+                const float on = s < nsteps ? 1.0f : 0.0f;
+                const float sa = h2f((uint16_t)st.sa[k]) * on, sb = h2f((uint16_t)st.sb[k]) * on;
+                const int zsh = 4 * (((sc * kStepCodes) >> lg) & 7);
+                // the 4-bit zero becomes a float through the 2^23 magic number
                 const float za = __uint_as_float(0x4B000000u | ((st.za >> zsh) & 15u)) - 8388608.0f;
                 const float zb = __uint_as_float(0x4B000000u | ((st.zb >> zsh) & 15u)) - 8388608.0f;
-                const float x0 = m0 < M ? xs0[s] : 0.f;
-                const float x1 = m1 < M ? xs1[s] : 0.f;
-                y[0] = fmaf(sa, fmaf(fmaf(d16[0], 0.0625f, d1[0]), 16777216.0f, -za * x0), y[0]);
-                y[1] = fmaf(sa, fmaf(fmaf(d16[1], 0.0625f, d1[1]), 16777216.0f, -za * x1), y[1]);
-                y[2] = fmaf(sb, fmaf(fmaf(d16[2], 0.0625f, d1[2]), 16777216.0f, -zb * x0), y[2]);
-                y[3] = fmaf(sb, fmaf(fmaf(d16[3], 0.0625f, d1[3]), 16777216.0f, -zb * x1), y[3]);
+                const float sa24 = sa * 16777216.0f, sb24 = sb * 16777216.0f;
+                const float x0 = xs0[sc] * xm0;
+                y[0] = fmaf(sa24, fmaf(d16[0], 0.0625f, d1[0]), fmaf(-sa * za, x0, y[0]));
+                y[2] = fmaf(sb24, fmaf(d16[2], 0.0625f, d1[2]), fmaf(-sb * zb, x0, y[2]));
+                if (!ONE) {
+                    const float x1 = xs1[sc] * xm1;
+                    y[1] = fmaf(sa24, fmaf(d16[1], 0.0625f, d1[1]), fmaf(-sa * za, x1, y[1]));
+                    y[3] = fmaf(sb24, fmaf(d16[3], 0.0625f, d1[3]), fmaf(-sb * zb, x1, y[3]));
+                }
             }
             if (u0 + i + kGemvDepth < U) load_next(buf[i]);
             if (++c_i == per) {
-                // end of a row group: combine the 8 warps' partial sums in a fixed order
+                // end of an iteration: combine the KS partial sums of each row in a fixed order
                 float* slot = part + (c_r & 1) * (kGemvWarps * kGemvRows * 8);
                 float* pw = slot + warp * kGemvRows * 8;
                 pw[g * 8 + 2 * t] = y[0];
@@ -272,18 +317,350 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
                 pw[(g + 8) * 8 + 2 * t + 1] = y[3];
                 y[0] = y[1] = y[2] = y[3] = 0.f;
                 __syncthreads();
-                if (threadIdx.x < kGemvRows * 8) {
-                    const int r = threadIdx.x >> 3, m = threadIdx.x & 7;
+                for (int o = threadIdx.x; o < RPI * kGemvRows * 8; o += kGemvThreads) {
+                    const int sb2 = o / (kGemvRows * 8);
+                    const int e = o - sb2 * (kGemvRows * 8);
+                    const int r = e >> 3, m = e & 7;
                     float acc = 0.f;
-#pragma unroll
-                    for (int w = 0; w < kGemvWarps; ++w) acc += slot[w * kGemvRows * 8 + threadIdx.x];
-                    const int n = c_rg * kGemvRows + r;
+                    for (int w = 0; w < KS; ++w) acc += slot[(sb2 * KS + w) * kGemvRows * 8 + e];
+                    const int n = (c_it * RPI + sb2) * kGemvRows + r;
                     if (m < M && n < N) Y[(size_t)m * N + n] = f2h_rn(acc);
                 }
                 c_i = 0;
-                c_rg += gridDim.x;
+                c_it += gridDim.x;
                 ++c_r;
             }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// TMA-staged GEMV for N % 16 == 0 (every real layer): the same arithmetic as
+// gemv_mma_kernel with a different data path.
+//   * Weights reach shared memory through one 3-D tensor TMA copy per stage
+//     (16 rows x 2048 codes = 16 KB) issued by a producer warp into a 4-stage ring.
+//     The 3-D view {16 words, rows, 128-code blocks} lands a stage as
+//     [block][row][64 B], so the two rows a quarter-warp reads are adjacent and the
+//     shared loads are conflict-free (row-major stages gave 8-way conflicts).
+//     Measured on B200: 16 per-row bulk copies per stage cap the copy rate near
+//     2 TB/s; one tensor copy per stage does not.
+//   * Scales and zero words of a row group arrive through two bulk copies into a raw
+//     parameter buffer; a converter warp turns them into fp32 pairs
+//     (scale16 * 2^24, scale16 * zero) per (row, group), so the consumers' fold is
+//     two shared loads and three FMAs per row.
+//   * The 8 consumer warps run only the decode, the MMAs and the fold, each taking
+//     1/8 of a stage's k-steps; no register ring, no global address math, no
+//     predication.  Every wait is bounded.
+// ---------------------------------------------------------------------------
+
+constexpr int kTmaConsumers = 8;                            // consumer warps
+constexpr int kTmaThreads = (kTmaConsumers + 2) * 32;       // + producer warp + converter warp
+constexpr int kTmaStages = 4;
+constexpr int kTmaKC = 2048;                                // codes per row per stage
+constexpr int kTmaBlkBytes = kGemvRows * 64;               // one 128-code block of 16 rows
+constexpr int kTmaStageBytes = (kTmaKC / 128) * kTmaBlkBytes;
+
+struct GemvTmaSmem {
+    int K, M, nsteps, ng, nzw;
+    __host__ __device__ GemvTmaSmem(int M_, int K_, int G) : K(K_), M(M_) {
+        nsteps = K / (32 * gemv_words_per_thread(G));
+        ng = K / G;
+        nzw = (ng + 7) / 8;
+    }
+    static __host__ __device__ size_t al16(size_t x) { return (x + 15) & ~(size_t)15; }
+    __host__ __device__ size_t raw_scale_bytes() const { return (size_t)kGemvRows * ng * 2; }
+    __host__ __device__ size_t raw_zero_bytes() const { return (size_t)kGemvRows * nzw * 4; }
+    __host__ __device__ size_t raw_stride() const { return al16(raw_scale_bytes()) + al16(raw_zero_bytes()); }
+    __host__ __device__ size_t cvt_stride() const { return (size_t)kGemvRows * ng * 8; }
+    __host__ __device__ size_t raw() const { return (size_t)kTmaStages * kTmaStageBytes; }
+    __host__ __device__ size_t cvt() const { return raw() + 2 * raw_stride(); }
+    __host__ __device__ size_t x() const { return al16(cvt() + 2 * cvt_stride()); }
+    __host__ __device__ size_t xsum() const { return x() + (size_t)M * GemvSmem::x_pitch(K); }
+    __host__ __device__ size_t part() const { return al16(xsum() + (size_t)M * nsteps * 4); }
+    __host__ __device__ size_t zero() const { return part() + (size_t)2 * kTmaConsumers * kGemvRows * 8 * 4; }
+    __host__ __device__ size_t bars() const { return (zero() + 64 + 7) & ~(size_t)7; }
+    // full[S], empty[S], pfull[2], rawfree[2], pready[2], pempty[2]
+    __host__ __device__ size_t bytes() const { return bars() + (2 * kTmaStages + 8) * 8; }
+};
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(sm100::smem_u32(dst)), "l"(src), "r"(bytes), "r"(sm100::smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float ldsf(uint32_t a) { return __uint_as_float(lds32(a)); }
+
+template <int WT>
+__device__ __forceinline__ void lds_words(uint32_t a, uint32_t* w) {
+    if constexpr (WT == 4) {
+        const uint4 v = lds128(a);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else if constexpr (WT == 2) {
+        const uint2 v = lds64(a);
+        w[0] = v.x; w[1] = v.y;
+    } else {
+        w[0] = lds32(a);
+    }
+}
+
+template <int WT, bool ONE>
+__global__ void __launch_bounds__(kTmaThreads, 2)
+gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __restrict__ X, int M,
+                const uint16_t* __restrict__ scales, const uint32_t* __restrict__ qzeros, int N, int K, int G,
+                int zero_point, uint16_t* __restrict__ Y) {
+    using namespace sm100;
+    constexpr int kStepCodes = 32 * WT;
+    constexpr int kStepsPerStage = kTmaKC / kStepCodes;
+    constexpr int kStepsPerWarp = kStepsPerStage / kTmaConsumers;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const GemvTmaSmem L(M, K, G);
+    const int nsteps = L.nsteps, ng = L.ng, nzw = L.nzw;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const bool zp = zero_point != 0;
+    const int n_rg = N / kGemvRows;
+    const int my_rg = blockIdx.x < n_rg ? (n_rg - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int nchunks = (K + kTmaKC - 1) / kTmaKC;
+    const int lg = 31 - __clz(G);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars());
+    uint64_t* empty = full + kTmaStages;
+    uint64_t* pfull = empty + kTmaStages;      // raw parameters landed
+    uint64_t* rawfree = pfull + 2;             // converter done with the raw buffer
+    uint64_t* pready = rawfree + 2;            // converted parameters ready
+    uint64_t* pempty = pready + 2;             // consumers done with the converted parameters
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kTmaStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kTmaConsumers);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&pfull[i], 1);
+            mbar_init(&rawfree[i], 1);
+            mbar_init(&pready[i], 1);
+            mbar_init(&pempty[i], kTmaConsumers);
+        }
+        mbar_fence_init();
+        prefetch_tensormap(&tmap_q);
+    }
+    __syncthreads();
+
+    if (warp == kTmaConsumers) {
+        // ---------------- producer (weights, scales and zeros do not depend on X) ----------------
+        if (lane == 0) {
+            int stage = 0;
+            bool ok = true;
+            const uint32_t pbytes = (uint32_t)(L.raw_scale_bytes() + (zp ? L.raw_zero_bytes() : 0));
+            for (int rgi = 0; rgi < my_rg && ok; ++rgi) {
+                const int r0 = (blockIdx.x + rgi * gridDim.x) * kGemvRows;
+                const int pb = rgi & 1;
+                if (rgi >= 2) ok = mbar_wait(&rawfree[pb], ((rgi >> 1) - 1) & 1);
+                if (!ok) break;
+                uint8_t* raw = smem + L.raw() + pb * L.raw_stride();
+                mbar_arrive_expect_tx(&pfull[pb], pbytes);
+                bulk_g2s(raw, scales + (size_t)r0 * ng, (uint32_t)L.raw_scale_bytes(), &pfull[pb]);
+                if (zp)
+                    bulk_g2s(raw + L.al16(L.raw_scale_bytes()), qzeros + (size_t)r0 * nzw,
+                             (uint32_t)L.raw_zero_bytes(), &pfull[pb]);
+                for (int c = 0; c < nchunks && ok; ++c, ++stage) {
+                    const int st = stage % kTmaStages;
+                    if (stage >= kTmaStages && !(ok = mbar_wait(&empty[st], ((stage / kTmaStages) - 1) & 1))) break;
+                    // box {16 words, 16 rows, 16 blocks}; blocks past K are filled with zeros
+                    mbar_arrive_expect_tx(&full[st], kTmaStageBytes);
+                    tma_load_3d(smem + (size_t)st * kTmaStageBytes, &tmap_q, &full[st], 0, r0, c * (kTmaKC / 128));
+                }
+            }
+            // drain: copies in flight must land before the CTA exits
+            for (int s2 = stage - 1; s2 >= 0 && s2 >= stage - kTmaStages; --s2)
+                mbar_wait(&full[s2 % kTmaStages], (s2 / kTmaStages) & 1);
+        }
+        return;
+    }
+    if (warp == kTmaConsumers + 1) {
+        // ---------------- converter: raw scales/zeros -> (scale16 * 2^24, scale16 * zero) ----------------
+        bool ok = true;
+        for (int rgi = 0; rgi < my_rg && ok; ++rgi) {
+            const int pb = rgi & 1;
+            ok = mbar_wait(&pfull[pb], (rgi >> 1) & 1);
+            if (ok && rgi >= 2) ok = mbar_wait(&pempty[pb], ((rgi >> 1) - 1) & 1);
+            if (!ok) break;
+            const uint8_t* raw = smem + L.raw() + pb * L.raw_stride();
+            const uint16_t* rs = reinterpret_cast<const uint16_t*>(raw);
+            const uint32_t* rz = reinterpret_cast<const uint32_t*>(raw + L.al16(L.raw_scale_bytes()));
+            float2* cv = reinterpret_cast<float2*>(smem + L.cvt() + pb * L.cvt_stride());
+            for (int e = lane; e < kGemvRows * ng; e += 32) {
+                const int r = e / ng, grp = e - r * ng;
+                const float sc = h2f(rs[e]);
+                const float z = zp ? (float)((rz[r * nzw + (grp >> 3)] >> (4 * (grp & 7))) & 15u) : 8.0f;
+                cv[e] = make_float2(sc * 16777216.0f, sc * z);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&rawfree[pb]);
+                mbar_arrive(&pready[pb]);
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumers: stage X (permuted) and its per-step sums ----------------
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const size_t pitch = GemvSmem::x_pitch(K);
+    uint8_t* xs = smem + L.x();
+    float* xsum = reinterpret_cast<float*>(smem + L.xsum());
+    const int kw = K >> 3;
+    constexpr int kCons = kTmaConsumers * 32;
+    for (int u0 = threadIdx.x; u0 < M * kw; u0 += kCons * 4) {
+        uint4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int u = u0 + i * kCons;
+            if (u < M * kw) {
+                const int m = u / kw;
+                v[i] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)m * K + (u - m * kw) * 8));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int u = u0 + i * kCons;
+            if (u < M * kw) {
+                const int m = u / kw;
+                const int word = u - m * kw;
+                uint4 p;
+                p.x = __byte_perm(v[i].x, v[i].z, 0x5410);
+                p.y = __byte_perm(v[i].y, v[i].w, 0x5410);
+                p.z = __byte_perm(v[i].x, v[i].z, 0x7632);
+                p.w = __byte_perm(v[i].y, v[i].w, 0x7632);
+                const int s = word / (4 * WT);
+                const int r = word - s * 4 * WT;
+                const int tt = r / WT, j = r - tt * WT;
+                *reinterpret_cast<uint4*>(xs + m * pitch + ((size_t)(s * WT + j) * 4 + tt) * 16) = p;
+            }
+        }
+    }
+    if (threadIdx.x < 16) reinterpret_cast<uint32_t*>(smem + L.zero())[threadIdx.x] = 0u;
+    asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    for (int u = threadIdx.x; u < M * nsteps; u += kCons) {
+        const int m = u / nsteps;
+        const int s = u - m * nsteps;
+        const uint4* xr = reinterpret_cast<const uint4*>(xs + m * pitch) + (size_t)s * WT * 4;
+        float acc = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4 * WT; ++i) {
+            const uint4 v = xr[i];
+            const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc += h2f(h[e]);
+        }
+        xsum[u] = acc;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
+
+    // ---------------- consumers: stream the stages ----------------
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t sbase = smem_u32(smem);
+    // lane's B column: X row g, or the zero row when g >= M
+    const uint32_t xrow = g < M ? smem_u32(xs + g * pitch) + t * 16 : smem_u32(smem + L.zero()) + t * 16;
+    const uint32_t xstep = g < M ? 64u : 0u;
+    const int m0 = 2 * t, m1 = 2 * t + 1;
+    const uint32_t xs0 = smem_u32(xsum + (m0 < M ? m0 : 0) * nsteps);
+    const uint32_t xs1 = smem_u32(xsum + (m1 < M ? m1 : 0) * nsteps);
+    const float xm0 = m0 < M ? 1.0f : 0.0f, xm1 = m1 < M ? 1.0f : 0.0f;
+    const uint32_t cbase = smem_u32(smem + L.cvt());
+    float* part = reinterpret_cast<float*>(smem + L.part());
+    // word w of row r in block b of a stage sits at b * kTmaBlkBytes + r * 64 + w * 4
+    const uint32_t wrow_a = (uint32_t)(g * 64 + t * WT * 4);
+    const uint32_t wrow_b = wrow_a + 8 * 64;
+    constexpr int kStepsPerBlk = 4 / WT;      // k-steps per 128-code block
+    const uint32_t prow_a = (uint32_t)(g * ng * 8), prow_b = (uint32_t)((g + 8) * ng * 8);
+
+    int stage = 0;
+    bool ok = true;
+    for (int rgi = 0; rgi < my_rg; ++rgi) {
+        const int pb = rgi & 1;
+        ok = ok && mbar_wait(&pready[pb], (rgi >> 1) & 1);
+        const uint32_t cv = cbase + (uint32_t)(pb * L.cvt_stride());
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c = 0; c < nchunks; ++c, ++stage) {
+            const int st = stage % kTmaStages;
+            ok = ok && mbar_wait(&full[st], (stage / kTmaStages) & 1);
+            const uint32_t sb = sbase + (uint32_t)(st * kTmaStageBytes);
+#pragma unroll
+            for (int q = 0; q < kStepsPerWarp; ++q) {
+                const int ks = warp * kStepsPerWarp + q;          // k-step inside the stage
+                const int s = c * kStepsPerStage + ks;            // k-step inside the row
+                if (!ok || s >= nsteps) break;
+                uint32_t wa[WT], wb[WT];
+                const uint32_t koff = (uint32_t)((ks / kStepsPerBlk) * kTmaBlkBytes + (ks % kStepsPerBlk) * WT * 16);
+                lds_words<WT>(sb + wrow_a + koff, wa);
+                lds_words<WT>(sb + wrow_b + koff, wb);
+                float d1[4], d16[4];
+#pragma unroll
+                for (int j = 0; j < WT; ++j) {
+                    const uint4 b = lds128(xrow + (uint32_t)(s * WT + j) * xstep);
+                    const uint32_t wa8 = wa[j] >> 8, wb8 = wb[j] >> 8;
+                    if (j == 0) {
+                        mma_16816_first(d1, wa[j] & 0x000F000Fu, wb[j] & 0x000F000Fu, wa8 & 0x000F000Fu,
+                                        wb8 & 0x000F000Fu, b.x, b.y);
+                        mma_16816_first(d16, wa[j] & 0x00F000F0u, wb[j] & 0x00F000F0u, wa8 & 0x00F000F0u,
+                                        wb8 & 0x00F000F0u, b.z, b.w);
+                    } else {
+                        mma_16816(d1, wa[j] & 0x000F000Fu, wb[j] & 0x000F000Fu, wa8 & 0x000F000Fu,
+                                  wb8 & 0x000F000Fu, b.x, b.y);
+                        mma_16816(d16, wa[j] & 0x00F000F0u, wb[j] & 0x00F000F0u, wa8 & 0x00F000F0u,
+                                  wb8 & 0x00F000F0u, b.z, b.w);
+                    }
+                }
+                // fold: y += (scale16 2^24) (D1 + D16/16) - (scale16 z) sum_k x
+                const int grp = (s * kStepCodes) >> lg;
+                const uint2 pa = lds64(cv + prow_a + grp * 8);
+                const uint2 pbv = lds64(cv + prow_b + grp * 8);
+                const float x0 = ldsf(xs0 + s * 4) * xm0;
+                y[0] = fmaf(__uint_as_float(pa.x), fmaf(d16[0], 0.0625f, d1[0]), fmaf(-__uint_as_float(pa.y), x0, y[0]));
+                y[2] = fmaf(__uint_as_float(pbv.x), fmaf(d16[2], 0.0625f, d1[2]), fmaf(-__uint_as_float(pbv.y), x0, y[2]));
+                if (!ONE) {
+                    const float x1 = ldsf(xs1 + s * 4) * xm1;
+                    y[1] = fmaf(__uint_as_float(pa.x), fmaf(d16[1], 0.0625f, d1[1]), fmaf(-__uint_as_float(pa.y), x1, y[1]));
+                    y[3] = fmaf(__uint_as_float(pbv.x), fmaf(d16[3], 0.0625f, d1[3]), fmaf(-__uint_as_float(pbv.y), x1, y[3]));
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        // row group done: parameters released; combine the 8 partial sums in a fixed order
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pempty[pb]);
+        float* slot = part + pb * (kTmaConsumers * kGemvRows * 8);
+        float* pw = slot + warp * kGemvRows * 8;
+        pw[g * 8 + 2 * t] = y[0];
+        pw[g * 8 + 2 * t + 1] = y[1];
+        pw[(g + 8) * 8 + 2 * t] = y[2];
+        pw[(g + 8) * 8 + 2 * t + 1] = y[3];
+        asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
+        if (threadIdx.x < kGemvRows * 8) {
+            const int r = threadIdx.x >> 3, m = threadIdx.x & 7;
+            float acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < kTmaConsumers; ++w) acc += slot[w * kGemvRows * 8 + threadIdx.x];
+            const int n = (blockIdx.x + rgi * gridDim.x) * kGemvRows + r;
+            if (m < M) Y[(size_t)m * N + n] = f2h_rn(acc);
         }
     }
 }
