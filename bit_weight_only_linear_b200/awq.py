@@ -38,6 +38,9 @@ SIGNATURES = {
     "awq_scale_search": (ctypes.c_int, [_u16p, ctypes.c_int32, _u16p, ctypes.c_int32, ctypes.c_int32,
                                         QuantConfig, ctypes.c_int32, _u16p, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "awq_scale_search_noalloc": (ctypes.c_int, [_u16p, ctypes.c_int32, _u16p, ctypes.c_int32, ctypes.c_int32,
+                                                QuantConfig, ctypes.c_int32, _u16p, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p]),
     "awq_fold_inverse_scale": (ctypes.c_int, [_u16p, _u16p, ctypes.c_int32, ctypes.c_int32, _u16p,
                                               ctypes.c_void_p]),
     "awq_linear_gemv": (ctypes.c_int, [_u16p, ctypes.c_int32, _u32p, _u16p, _u32p, ctypes.c_int32,
@@ -195,6 +198,23 @@ def scale_search(X: torch.Tensor, W: torch.Tensor, group_size: int = 128, zero_p
         _dev(s_out, "s_out", _F16), losses.data_ptr(), best.data_ptr(), workspace.data_ptr(),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check("awq_scale_search", st)
+    return s_out, losses, best
+
+
+def scale_search_noalloc(X: torch.Tensor, W: torch.Tensor, group_size: int = 128, zero_point: bool = True,
+                         n_grid: int = 20, stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """awq_scale_search_noalloc: the scale search on the library's fixed scratch (for
+    callers that cannot allocate device memory).  Returns (s*, losses, best index) on
+    device; the output tensors here are allocated by torch only for convenience."""
+    M, K = X.shape
+    N = W.shape[0]
+    s_out = torch.empty(K, dtype=torch.float16, device=X.device)
+    losses = torch.empty(n_grid, dtype=torch.float64, device=X.device)
+    best = torch.empty(1, dtype=torch.int32, device=X.device)
+    st = load_library().awq_scale_search_noalloc(
+        _dev(X, "X", _F16), M, _dev(W, "W", _F16), N, K, config(group_size, zero_point), n_grid,
+        _dev(s_out, "s_out", _F16), losses.data_ptr(), best.data_ptr(), _stream(stream))
+    _check("awq_scale_search_noalloc", st)
     return s_out, losses, best
 
 

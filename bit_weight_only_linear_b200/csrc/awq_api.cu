@@ -186,6 +186,48 @@ awq_status dispatch_gemv(const uint16_t* X, int M, const uint32_t* qweight, cons
     }
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for awq_scale_search_noalloc.  Some callers cannot allocate device
+// memory at the point where they quantise (an allocator-less runtime, a memory
+// pool that is already fully carved up, a process that must not grow its
+// footprint after start-up), so this entry point keeps its scratch in a
+// file-scope device array instead of asking for a workspace.  Every device that
+// loads the library holds these bytes until the process exits.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = (size_t)12 << 20;   // 12 MiB
+constexpr int kNoAllocMaxK = 16384;
+constexpr int kNoAllocMaxM = 1 << 20;
+
+struct NoAllocScratch {
+    bool ready = false;
+    void* ptr = nullptr;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of the scratch array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+awq_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    NoAllocScratch& s = g_noalloc[dev];
+    if (!s.ready) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return AWQ_ERR_CUDA;
+        s.ptr = p;
+        s.ready = true;
+    }
+    *out = s.ptr;
+    return AWQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -279,6 +321,26 @@ awq_status awq_scale_search(const uint16_t* X, int32_t M, const uint16_t* W, int
     if (!device_info(d)) return AWQ_ERR_CUDA;
     return run_scale_search(X, M, W, N, K, cfg.q_group_size, cfg.zero_point, n_grid, s_out, losses_out,
                             best_index_out, ws, (cudaStream_t)stream, d.sms);
+}
+
+awq_status awq_scale_search_noalloc(const uint16_t* X, int32_t M, const uint16_t* W, int32_t N, int32_t K,
+                                    awq_quant_config cfg, int32_t n_grid, uint16_t* s_out, double* losses_out,
+                                    int32_t* best_index_out, void* stream) {
+    awq_status st = check_config(cfg);
+    if (st != AWQ_OK) return st;
+    st = check_shape(N, K, cfg);
+    if (st != AWQ_OK) return st;
+    if (M <= 0 || n_grid < 1 || n_grid > kSearchMaxGrid) return AWQ_ERR_INVALID_ARG;
+    if (!X || !W || !s_out) return AWQ_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(s_out)) return AWQ_ERR_INVALID_ARG;
+    if (K > kNoAllocMaxK || M > kNoAllocMaxM) return AWQ_ERR_UNSUPPORTED;   // beyond the fixed scratch
+    void* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != AWQ_OK) return st;
+    const ChunkedSearchLayout L = chunked_search_layout(scratch, kNoAllocScratchBytes, M, N, K);
+    if (L.nc <= 0) return AWQ_ERR_UNSUPPORTED;
+    return run_scale_search_chunked(X, M, W, N, K, cfg.q_group_size, cfg.zero_point, n_grid, s_out, losses_out,
+                                    best_index_out, L, (cudaStream_t)stream);
 }
 
 awq_status awq_device_error(void* stream) {

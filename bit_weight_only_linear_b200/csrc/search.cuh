@@ -369,4 +369,111 @@ inline awq_status run_scale_search(const uint16_t* X, int M, const uint16_t* W, 
     return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// Same search over caller-provided scratch of bounded size: one alpha and one
+// chunk of output channels at a time, the chunk's tile sums added to the running
+// loss in a fixed order (deterministic).  Used by awq_scale_search_noalloc.
+// ---------------------------------------------------------------------------
+
+// losses[0] = (first ? 0 : losses[0]) + sum of the tile partials; * scale when last.
+__global__ void search_accum_kernel(const double* __restrict__ partial, int tiles, int first, int last, double scale,
+                                    double* __restrict__ loss) {
+    __shared__ double sh[256];
+    double acc = 0.0;
+    for (int i = threadIdx.x; i < tiles; i += 256) acc += partial[i];
+    sh[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if (threadIdx.x < w) sh[threadIdx.x] += sh[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        double v = (first ? 0.0 : *loss) + sh[0];
+        if (last) v *= scale;
+        *loss = v;
+    }
+}
+
+struct ChunkedSearchLayout {
+    double* colsum;      // [K]
+    uint16_t* s_all;     // [kSearchMaxGrid][K]
+    double* losses;      // [kSearchMaxGrid]
+    double* partial;     // [partial_cap]
+    int32_t* row_exp;    // [nc]
+    uint16_t* dw;        // [nc][2*Kp]
+    int nc;              // output channels per chunk (multiple of kSearchTileN), 0 if it does not fit
+    size_t partial_cap;
+};
+
+inline ChunkedSearchLayout chunked_search_layout(void* base, size_t bytes, int M, int N, int K) {
+    ChunkedSearchLayout L = {};
+    char* b = static_cast<char*>(base);
+    size_t off = 0;
+    auto take = [&](size_t n) {
+        char* p = b + off;
+        off += align256(n);
+        return p;
+    };
+    L.colsum = reinterpret_cast<double*>(take((size_t)K * 8));
+    L.s_all = reinterpret_cast<uint16_t*>(take((size_t)kSearchMaxGrid * K * 2));
+    L.losses = reinterpret_cast<double*>(take((size_t)kSearchMaxGrid * 8));
+    L.partial_cap = 32768;   // doubles
+    L.partial = reinterpret_cast<double*>(take(L.partial_cap * 8));
+    if (off >= bytes) return L;
+    const size_t per_row = (size_t)2 * search_kp(K) * 2 + 4;      // dW row + its exponent
+    size_t nc = (bytes - off - 512) / per_row;
+    nc = nc / kSearchTileN * kSearchTileN;
+    const size_t n_cap = (size_t)ceil_div(N, kSearchTileN) * kSearchTileN;
+    if (nc > n_cap) nc = n_cap;
+    const size_t mt = (size_t)ceil_div(M, kSearchTileM);
+    while (nc > 0 && mt * (nc / kSearchTileN) > L.partial_cap) nc -= kSearchTileN;
+    L.nc = (int)nc;
+    if (nc == 0) return L;
+    L.row_exp = reinterpret_cast<int32_t*>(take(nc * 4));
+    L.dw = reinterpret_cast<uint16_t*>(take(nc * 2 * (size_t)search_kp(K) * 2));
+    if (off > bytes) L.nc = 0;
+    return L;
+}
+
+inline awq_status run_scale_search_chunked(const uint16_t* X, int M, const uint16_t* W, int N, int K, int G, int zp,
+                                           int n_grid, uint16_t* s_out, double* losses_out, int32_t* best_out,
+                                           const ChunkedSearchLayout& L, cudaStream_t st) {
+    if (L.nc <= 0) return AWQ_ERR_UNSUPPORTED;
+    if (cudaMemsetAsync(L.colsum, 0, (size_t)K * 8, st) != cudaSuccess) return AWQ_ERR_CUDA;
+    abs_colsum_kernel<<<dim3(ceil_div(K / 8, 128), (unsigned)min(M, 64)), 128, 0, st>>>(X, M, K, L.colsum);
+    scales_for_alphas_kernel<<<dim3(ceil_div(K, 256), n_grid), 256, 0, st>>>(L.colsum, M, K, n_grid, L.s_all);
+    if (cudaGetLastError() != cudaSuccess) return AWQ_ERR_CUDA;
+    const size_t dsm = (size_t)K * 4 + 32 * 4;
+    if (dsm > 48 * 1024 &&
+        cudaFuncSetAttribute(search_delta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm) != cudaSuccess)
+        return AWQ_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(search_sumsq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SearchGemmCfg::kSmemBytes) != cudaSuccess)
+        return AWQ_ERR_CUDA;
+    CUtensorMap tx;
+    if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)M, (uint64_t)K, kSearchTileM, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return AWQ_ERR_CUDA;
+    const int mt = ceil_div(M, kSearchTileM);
+    const double inv_mn = 1.0 / ((double)M * (double)N);
+    for (int a = 0; a < n_grid; ++a) {
+        for (int n0 = 0; n0 < N; n0 += L.nc) {
+            const int nc = min(L.nc, N - n0);
+            search_delta_kernel<<<dim3(nc, 1), kQuantThreads, dsm, st>>>(W + (size_t)n0 * K, L.s_all + (size_t)a * K,
+                                                                        nc, K, G, zp, L.dw, L.row_exp);
+            CUtensorMap td;
+            if (!make_tmap_2d(&td, L.dw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)nc, (uint64_t)2 * search_kp(K),
+                              kSearchTileN, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+                return AWQ_ERR_CUDA;
+            const int ntc = ceil_div(nc, kSearchTileN);
+            search_sumsq_kernel<<<dim3(mt, ntc, 1), kSearchThreads, SearchGemmCfg::kSmemBytes, st>>>(
+                tx, td, M, nc, K, L.row_exp, L.partial);
+            search_accum_kernel<<<1, 256, 0, st>>>(L.partial, mt * ntc, n0 == 0, n0 + nc >= N, inv_mn, L.losses + a);
+            if (cudaGetLastError() != cudaSuccess) return AWQ_ERR_CUDA;
+        }
+    }
+    search_select_kernel<<<ceil_div(K, 256), 256, 0, st>>>(L.losses, n_grid, L.s_all, K, s_out, best_out, losses_out);
+    return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
 }  // namespace awq

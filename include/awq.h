@@ -151,6 +151,28 @@ awq_status awq_linear_gemm(const uint16_t* X, int32_t M, const uint32_t* qweight
                            awq_quant_config cfg, uint16_t* Y, void* ws, size_t ws_bytes,
                            void* stream);
 
+/*
+ * awq_scale_search without a workspace argument, for callers that cannot allocate
+ * device memory when they quantise (an allocator-less runtime, a memory pool that
+ * is already fully carved up, a process that must not grow after start-up).  The
+ * pages have no counterpart: this is a property of this library, not of the method.
+ *
+ * Scratch lives in a fixed 12 MiB device array inside the library; every device
+ * that loads the library holds it until the process exits.  The result is the one
+ * awq_scale_search defines; only the order in which the loss is summed differs
+ * (one alpha and one chunk of output channels at a time), so losses agree to
+ * rounding.  Limits: K <= 16384 and M <= 2^20 (larger sizes return
+ * AWQ_ERR_UNSUPPORTED before anything is launched); any N.
+ * The first call on a device looks up the array's device address (with that device
+ * current); make that first call before any stream capture.  All calls on a
+ * device share the array and it keeps the last call's contents: calls that can
+ * overlap on the GPU (different streams, no ordering) race and must not be made.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+awq_status awq_scale_search_noalloc(const uint16_t* X, int32_t M, const uint16_t* W, int32_t N, int32_t K,
+                                    awq_quant_config cfg, int32_t n_grid, uint16_t* s_out, double* losses_out,
+                                    int32_t* best_index_out, void* stream);
+
 /* Workspace bytes an operation needs for the given sizes (0 = none). */
 size_t awq_workspace_bytes(int32_t op, int32_t M, int32_t N, int32_t K, awq_quant_config cfg);
 
