@@ -5,8 +5,10 @@
 Headline (`value`): decode GEMV throughput over one Mistral-7B-shaped layer at M=1
 (q/k/v/o 4096->4096/1024/1024/4096, gate/up 4096->14336, down 14336->4096), group 128,
 zero point on, in GB/s of algorithmic bytes (packed codes + fp16 scales + packed zeros
-+ x + y).  One step = one pass over the seven linears, each from a different copy of
-the layer's weights so that every step reads HBM (4 rotated copies, 454 MB > 3x L2).
++ x + y).  One step = one pass over the layer with q/k/v and gate/up fused (their
+weights concatenated row-wise: 4 dependent launches, the same bytes), each from a
+different copy of the layer's weights so that every step reads HBM (4 rotated copies,
+454 MB > 3x L2).  The seven-launch (unfused) number is reported beside it.
 The same line also measures the other rows of the path:
   gemm         tcgen05 W4A16 GEMM on Llama-70B-shaped prefill linears at M=2048 (TFLOP/s)
   quantize     awq_quantize_pack on the 4096x4096 layer (GB/s)
@@ -37,7 +39,7 @@ G = 128
 ZP = True
 ROTATIONS = 4
 METRIC = "W4A16 linear: GEMV HBM GB/s (% of peak); GEMM TFLOPS (% of fp16 peak)"
-WORKLOAD = "mistral7b-layer-decode-gemv-m1-g128-zp"
+WORKLOAD = "mistral7b-layer-decode-gemv-m1-g128-zp-fused-qkv-gateup"
 
 
 def packed_bytes(N: int, K: int, g: int = G, zp: bool = ZP) -> int:
@@ -177,11 +179,13 @@ def _max_over_ranks(world, value_ms):
     return float(t.item())
 
 
-def build_decode_layer(awq, torch, seed_offset):
-    """Quantise the 7 Mistral linears on the GPU; return per-linear packed tensors
-    (ROTATIONS copies) and inputs."""
+def build_decode_layer(awq, torch, seed_offset, fused=False):
+    """Quantise the Mistral linears on the GPU (7, or 4 with q/k/v and gate/up
+    concatenated); return per-linear packed tensors (ROTATIONS copies) and inputs."""
     layers = []
-    for name, W, X in inputs.layer_inputs(inputs.MISTRAL_7B_LAYER, 1, 0.02, seed_offset):
+    src = (inputs.fused_layer_inputs(1, 0.02, seed_offset) if fused
+           else inputs.layer_inputs(inputs.MISTRAL_7B_LAYER, 1, 0.02, seed_offset))
+    for name, W, X in src:
         N, K = W.shape
         Wd = torch.from_numpy(W).cuda()
         q, sc, z = awq.quantize_pack(Wd, None, G, ZP)
@@ -359,10 +363,10 @@ def measure_search(awq, torch, reps=3):
 
 def cpu_baseline_sample(seconds: float = 12.0):
     """The oracle, as it stands, on a bounded sample of the decode workload: the first
-    256 output channels of each of the seven linears (fp64 dequantise + matmul)."""
+    256 output channels of each of the four fused linears (fp64 dequantise + matmul)."""
     from oracle import awq_oracle as O
     sample = []
-    for name, W, X in inputs.layer_inputs(inputs.MISTRAL_7B_LAYER, 1, 0.02):
+    for name, W, X in inputs.fused_layer_inputs(1, 0.02):
         Ws = W[:256]
         q, sc, z = O.quantize_pack(Ws, None, G, ZP)
         sample.append((X, q, sc, z, W.shape[1]))
@@ -382,7 +386,7 @@ def cpu_baseline_sample(seconds: float = 12.0):
     except Exception:
         cores = 1
     return {"value": round(nbytes * passes / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"first 256 output channels of each of the 7 linears ({nbytes} algorithmic bytes per "
+            "sample": f"first 256 output channels of each of the 4 fused linears ({nbytes} algorithmic bytes per "
                       f"pass), {passes} passes in {dt:.1f} s"}
 
 
@@ -397,8 +401,20 @@ def run_ours(args):
         dist.barrier()
     awq.load_library()
     peaks = read_peaks()
-    layers = build_decode_layer(awq, torch, seed_offset=rank * 100)
-    step_bytes = layer_bytes(inputs.MISTRAL_7B_LAYER, 1)
+    # the seven linears as separate launches (reported beside the headline)
+    unfused = build_decode_layer(awq, torch, seed_offset=rank * 100, fused=False)
+    step_bytes_7 = layer_bytes(inputs.MISTRAL_7B_LAYER, 1)
+    ms7, steps7 = time_decode(awq, torch, unfused, args.steps, args.warmup, world)
+    ms7 = _max_over_ranks(world, ms7)
+    launches7 = per_launch_gemv(awq, torch, unfused)
+    for L in unfused:
+        L.clear()
+    del unfused
+    torch.cuda.empty_cache()
+
+    # headline: the layer with q/k/v and gate/up fused (4 dependent launches per step)
+    layers = build_decode_layer(awq, torch, seed_offset=rank * 100, fused=True)
+    step_bytes = sum(linear_bytes(1, n, k) for _, k, n, _ in inputs.MISTRAL_7B_LAYER_FUSED)
 
     with ClockSampler(local) as clocks:
         ms, steps = time_decode(awq, torch, layers, args.steps, args.warmup, world)
@@ -415,8 +431,13 @@ def run_ours(args):
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "peak_source": peaks["source"] + " (burst copy bandwidth)",
                 "per_linear_us": {n: round(t * 1e3, 2) for n, _, t in launches}}
+    unfused_obj = {"workload": "mistral7b-layer-decode-gemv-m1-g128-zp-unfused",
+                   "value": round(world * step_bytes_7 * steps7 / (ms7 * 1e-3) / 1e9, 1), "unit": "GB/s",
+                   "ms_per_step": round(ms7 / steps7, 5), "launches_per_step": 7,
+                   "per_linear_us": {n: round(t * 1e3, 2) for n, _, t in launches7}}
 
     e2e_steps = max(50, min(args.steps, 400))
+    # note: time_decode_e2e copies each fused linear's input once per step
     e2e_ms, h2d, d2h = time_decode_e2e(awq, torch, layers, e2e_steps)
     e2e_ms = _max_over_ranks(world, e2e_ms)
     e2e = {"value": round(world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
@@ -446,12 +467,16 @@ def run_ours(args):
                 "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms / steps, 5),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u4-f16-f32acc",
                 "data": "synthetic (seeded fp16 N(0,0.02^2) weights, N(0,1) activations with 1% x20 channels)",
-                "config": {"workload": WORKLOAD, "linears": [f"{n}:{k}->{nn}" for n, k, nn in inputs.MISTRAL_7B_LAYER],
+                "config": {"workload": WORKLOAD,
+                           "linears": [f"{n}:{k}->{nn}" for n, k, nn, _ in inputs.MISTRAL_7B_LAYER_FUSED],
+                           "fusion": "q/k/v and gate/up weights concatenated row-wise (layer fusion); "
+                                     "same bytes as the seven linears",
                            "batch_m": 1, "group_size": G, "zero_point": ZP, "bytes_per_step": step_bytes,
                            "l2": f"weights rotated over {ROTATIONS} copies ({ROTATIONS * step_bytes / 1e6:.0f} MB > 3x L2)",
                            "timing": "CUDA graph of 4 layer passes, CUDA events, max over ranks"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": 7 * steps, "clocks": clk, **extra}
+                "gpu_launches": len(inputs.MISTRAL_7B_LAYER_FUSED) * steps, "clocks": clk,
+                "unfused": unfused_obj, **extra}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -460,13 +485,13 @@ def run_ours(args):
 
 def run_reference(args):
     """The oracle as it stands on the host cores: each step is a bounded sample of the
-    decode workload (256 output channels of each of the 7 linears)."""
+    decode workload (up to 256 output channels of each of the 4 fused linears)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     from oracle import awq_oracle as O
-    layer = list(inputs.layer_inputs(inputs.MISTRAL_7B_LAYER, 1, 0.02))
+    layer = list(inputs.fused_layer_inputs(1, 0.02))
 
     def make_sample(rows):
         out = []
@@ -502,7 +527,7 @@ def run_reference(args):
     except Exception:
         cores = 1
     value = nbytes * args.steps / dt / 1e9
-    sample_desc = f"first {rows} output channels of each of the 7 Mistral-7B linears per step"
+    sample_desc = f"first {rows} output channels of each of the 4 fused Mistral-7B linears per step"
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -513,6 +538,38 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """Profiling mode (no timing, no JSON): quantise the fused decode layer once, run
+    one warm-up pass and one pass of its four GEMV launches, run one launch of each
+    of the four Llama-70B prefill GEMMs, and exit.  ncu captures select kernels from
+    this with -k / -s / -c."""
+    import torch
+    from bit_weight_only_linear_b200 import awq, build
+    build.build()
+    awq.load_library()
+    torch.cuda.set_device(0)
+    layers = build_decode_layer(awq, torch, 0, fused=True)
+    for _ in range(2):
+        for L in layers:
+            q, sc, z = L["copies"][0]
+            awq.linear_gemv(L["x"], q, sc, z, G, ZP, out=L["y"])
+    torch.cuda.synchronize()
+    for L in layers:
+        L.clear()
+    torch.cuda.empty_cache()
+    if not args.skip_extra:
+        for i, (name, K, N) in enumerate(inputs.LLAMA_70B_FUSED):
+            W = torch.from_numpy(inputs.weights(N, K, 0.015, inputs.SEED_W + 30 + i)).cuda()
+            q, sc, z = awq.quantize_pack(W, None, G, ZP)
+            del W
+            X = torch.from_numpy(inputs.activations(2048, K, inputs.SEED_X + 30 + i, inputs.SEED_OUTLIER + 30)).cuda()
+            awq.linear_gemm(X, q, sc, z, G, ZP)
+            torch.cuda.synchronize()
+            del q, sc, z, X
+    awq.device_error()
+    print("profile run done", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -521,9 +578,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--skip-extra", action="store_true", help="headline decode measurement only")
     ap.add_argument("--skip-cpu", action="store_true", help="do not time the CPU oracle")
+    ap.add_argument("--profile", action="store_true",
+                    help="no timing: one pass of the decode layer and one launch of each prefill GEMM, for ncu")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.profile:
+        run_profile(args)
+        return
     if args.impl == "reference":
         if args.steps == 2000:
             args.steps = 20

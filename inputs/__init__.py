@@ -39,6 +39,16 @@ MISTRAL_7B_LAYER = (
     ("down_proj", 14336, 4096),
 )
 
+# The same layer with q/k/v and gate/up concatenated row-wise (one weight matrix and
+# one launch each), as the layer fusion of the AWQ inference path does:
+# (name, K, N, [names of the concatenated linears]).
+MISTRAL_7B_LAYER_FUSED = (
+    ("qkv_proj", 4096, 6144, ("q_proj", "k_proj", "v_proj")),
+    ("o_proj", 4096, 4096, ("o_proj",)),
+    ("gate_up_proj", 4096, 28672, ("gate_proj", "up_proj")),
+    ("down_proj", 14336, 4096, ("down_proj",)),
+)
+
 # Llama-70B-shaped prefill linears with q/k/v and gate/up fused:
 # (name, K, N).
 LLAMA_70B_FUSED = (
@@ -99,4 +109,17 @@ def layer_inputs(shapes, m: int, sigma: float, seed_offset: int = 0):
         w = weights(n, k, sigma, SEED_W + seed_offset + i)
         x = activations(m, k, SEED_X + seed_offset + i, SEED_OUTLIER + seed_offset)
         out.append((name, w, x))
+    return out
+
+
+def fused_layer_inputs(m: int, sigma: float, seed_offset: int = 0):
+    """Per fused linear (name, W, X): the weights of the concatenated linears of
+    MISTRAL_7B_LAYER (same seeds as layer_inputs) stacked row-wise, and the input of
+    the first of them (the concatenated linears share their input)."""
+    parts = {name: (w, x) for name, w, x in layer_inputs(MISTRAL_7B_LAYER, m, sigma, seed_offset)}
+    out = []
+    for name, k, n, members in MISTRAL_7B_LAYER_FUSED:
+        w = np.concatenate([parts[mname][0] for mname in members], axis=0)
+        assert w.shape == (n, k)
+        out.append((name, w, parts[members[0]][1]))
     return out

@@ -80,6 +80,18 @@ def test_gemv_mistral_layer_sampled(lib):
         assert_linear_close(y[:, rows], ref)
 
 
+def test_gemv_mistral_layer_fused_sampled(lib):
+    """The fused decode layer (q/k/v and gate/up concatenated) as benchmarked:
+    256 sampled output channels per fused linear against the oracle."""
+    rng = np.random.Generator(np.random.PCG64(6))
+    for name, W, X in inputs.fused_layer_inputs(1, 0.02):
+        N, K = W.shape
+        q, sc, z, dq = _packed(W, 128, True)
+        y = _run(lib, "gemv", X, dq, 128, True)
+        rows = np.sort(rng.choice(N, 256, replace=False))
+        assert_linear_close(y[:, rows], O.linear_rows(X, q, sc, z, K, 128, True, rows))
+
+
 GEMM_SMALL = [(1, 128, 128), (4, 256, 130), (16, 1024, 256), (17, 512, 384), (33, 256, 128),
               (64, 2048, 256), (100, 1024, 200), (128, 512, 128), (200, 256, 384), (256, 1024, 256),
               (300, 512, 136), (513, 256, 128)]
