@@ -11,11 +11,11 @@
 // is dequantised once per CTA and reused for BN tokens, so the dequant work per
 // multiply-add is 1/BN, and small token counts use a narrow MMA instead of padding.
 //
-// Warp roles (320 threads):
+// Warp roles (576 threads):
 //   warp 0      TMA producer: X tile [BN x 64] fp16 (128B swizzle) and the packed
 //               weight tile [128 x 8 words] per 64-channel k-block, into an S-stage ring.
 //   warp 1      allocates TMEM; one lane issues 4 tcgen05.mma (K = 16 each) per k-block.
-//   warps 2..9  dequantise: thread (row, half) turns 32 codes into fp16
+//   warps 2..17 dequantise: thread (row, quarter) turns 16 codes into fp16
 //               (q - z) * scale16 with mask/magic-number arithmetic and writes them in
 //               the 128B-swizzled K-major layout the MMA reads; afterwards they are the
 //               epilogue, reading the fp32 accumulator from TMEM and storing fp16 Y.
@@ -30,10 +30,11 @@
 
 namespace awq {
 
-constexpr int kGemmThreads = 320;
+constexpr int kDequantWarps = 16;
+constexpr int kGemmThreads = 64 + kDequantWarps * 32;   // TMA warp, MMA warp, dequant/epilogue warps
 constexpr int kGemmTileN = 128;      // output channels per CTA (MMA M)
 constexpr int kGemmKB = 64;          // input channels per k-block
-constexpr int kDequantThreads = 256;
+constexpr int kDequantThreads = kDequantWarps * 32;   // 4 threads per row, 16 codes each
 
 template <int BN>
 struct GemmCfg {
@@ -167,43 +168,58 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         }
     } else {
         // ---------------- dequantise, then epilogue ----------------
-        const int d = threadIdx.x - 64;           // 0..255
+        const int d = threadIdx.x - 64;           // 0..511
         const int row = d & (kGemmTileN - 1);
-        const int kh = d >> 7;                    // which 32 channels of the k-block
+        const int kq = d >> 7;                    // which 16 channels of the k-block
         const int n = n0 + row;
         const int ng = K / G;
         const int nzw = ceil_div(ng, 8);
         const bool zp = zero_point != 0;
+        const bool row_ok = n < N;
+        const uint16_t* srow = scales + (size_t)(row_ok ? n : 0) * ng;
+        const uint32_t* zrow = qzeros + (size_t)(row_ok ? n : 0) * nzw;
+        // scale and zero word of the thread's group, loaded one k-block ahead (raw; using a
+        // loaded value stalls on its load) and only when the group changes
+        int g_next = (kq * 16) / G;
+        uint32_t sc_next = row_ok ? __ldg(srow + g_next) : 0u;
+        uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_next >> 3)) : 0u;
+        int g_cur = -1;
+        uint32_t s2 = 0, zmagic = 0x64006400u, zneg16 = 0;
         bool ok = true;
         for (int kb = 0; kb < num_kb && ok; ++kb) {
             const int s = kb % C::kStages;
             const int a = kb % C::kABufs;
-            const int k = kb * kGemmKB + kh * 32;
-            // scale / zero of this thread's 32 channels (one group: G >= 32)
-            uint32_t s2 = 0, zmagic = 0x64006400u, zneg16 = 0;
-            const bool live = n < N && k < K;
-            if (live) {
-                const int g = k / G;
-                const uint32_t sc = __ldg(scales + (size_t)n * ng + g);
-                const uint32_t z = zp ? ((__ldg(qzeros + (size_t)n * nzw + (g >> 3)) >> (4 * (g & 7))) & 15u) : 8u;
+            const int k = kb * kGemmKB + kq * 16;
+            const bool live = row_ok && k < K;
+            if (live && g_next != g_cur) {
+                g_cur = g_next;
+                const uint32_t sc = sc_next;
+                const uint32_t z = zp ? ((zw_next >> (4 * (g_cur & 7))) & 15u) : 8u;
                 s2 = sc | (sc << 16);
                 const uint32_t zm = 0x6400u | z;                                   // 1024 + z
                 zmagic = zm | (zm << 16);
-                const uint32_t zn = __half_as_ushort(__float2half_rn(-(64.0f + (float)z)));
+                const uint32_t zn = 0xD000u | (z << 4) | 0x0400u;                  // fp16 -(64 + z): 2^6 * (1 + z/64)
                 zneg16 = zn | (zn << 16);
+            }
+            {   // prefetch the next k-block's group parameters if the group changes
+                const int kn = k + kGemmKB;
+                const int gn = kn / G;
+                if (row_ok && kn < K && gn != g_cur) {
+                    g_next = gn;
+                    sc_next = __ldg(srow + gn);
+                    if (zp) zw_next = __ldg(zrow + (gn >> 3));
+                }
             }
             if (kb >= C::kABufs) ok = mbar_wait(&aempty[a], ((kb / C::kABufs) - 1) & 1);
             ok = ok && mbar_wait(&full[s], (kb / C::kStages) & 1);
             if (!ok) break;
-            const uint4 packed =
-                *reinterpret_cast<const uint4*>(smem + C::kWOff + s * C::kWBytes + row * 32 + kh * 16);
+            const uint2 packed =
+                *reinterpret_cast<const uint2*>(smem + C::kWOff + s * C::kWBytes + row * 32 + kq * 8);
             uint8_t* atile = smem + C::kAOff + a * C::kABytes;
-            const uint32_t pw[4] = {packed.x, packed.y, packed.z, packed.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 v = live ? dequant_word(pw[i], zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4*>(atile + sw128_offset(row, kh * 4 + i)) = v;
-            }
+            const uint4 v0 = live ? dequant_word(packed.x, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+            const uint4 v1 = live ? dequant_word(packed.y, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(atile + sw128_offset(row, kq * 2)) = v0;
+            *reinterpret_cast<uint4*>(atile + sw128_offset(row, kq * 2 + 1)) = v1;
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&afull[a]);
@@ -211,10 +227,10 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         if (ok && mbar_wait(tfull, 0)) {
             tc_fence_after();
             const int q = warp & 3;                        // TMEM lane quarter this warp may access
-            const int set = (warp - 2) >> 2;               // 0: warps 2..5, 1: warps 6..9
-            const int cols = BN >= 32 ? BN / 2 : BN;
-            const int c_begin = BN >= 32 ? set * cols : 0;
-            if (BN >= 32 || set == 0) {
+            const int set = (warp - 2) >> 2;               // 0..3: four warps per lane quarter
+            const int cols = BN >= 64 ? BN / 4 : 16;
+            const int c_begin = set * cols;
+            if (c_begin < BN) {
                 const int nn = n0 + q * 32 + lane;
                 for (int c = c_begin; c < c_begin + cols; c += 16) {
                     uint32_t r[16];
