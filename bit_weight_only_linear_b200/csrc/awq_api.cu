@@ -122,7 +122,7 @@ awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const 
     return launch_status();
 }
 
-template <int WT, bool ONE>
+template <int G, bool ONE, bool FULL>
 awq_status launch_gemv_tma(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
                            const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
                            cudaStream_t st) {
@@ -136,7 +136,7 @@ awq_status launch_gemv_tma(const uint16_t* X, int M, const uint32_t* qweight, co
                       (uint64_t)K / 2, 64, 16, kGemvRows, kTmaKC / 128))
         return AWQ_ERR_CUDA;
     if (smem > (size_t)d.max_smem_optin) return AWQ_ERR_UNSUPPORTED;
-    auto kern = gemv_tma_kernel<WT, ONE>;
+    auto kern = gemv_tma_kernel<G, ONE, FULL>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return AWQ_ERR_CUDA;
     int occ = 0;
@@ -156,8 +156,7 @@ awq_status launch_gemv_tma(const uint16_t* X, int M, const uint32_t* qweight, co
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&lc, kern, tq, X, M, scales, qzeros, N, K, (int)cfg.q_group_size,
-                           (int)cfg.zero_point, Y) != cudaSuccess)
+    if (cudaLaunchKernelEx(&lc, kern, tq, X, M, scales, qzeros, N, K, (int)cfg.zero_point, Y) != cudaSuccess)
         return AWQ_ERR_CUDA;
     return launch_status();
 }
@@ -173,11 +172,17 @@ awq_status dispatch_gemv(const uint16_t* X, int M, const uint32_t* qweight, cons
     if (N % kGemvRows == 0 && K % 128 == 0 && (uintptr_t)scales % 16 == 0 &&
         (!cfg.zero_point || (uintptr_t)qzeros % 16 == 0) &&
         GemvTmaSmem(M, K, cfg.q_group_size).bytes() <= (size_t)d.max_smem_optin) {
+        const bool full = K % kTmaKC == 0;
+#define AWQ_GEMV_TMA(GG)                                                                                   \
+    return full ? launch_gemv_tma<GG, ONE, true>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s)          \
+                : launch_gemv_tma<GG, ONE, false>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s)
         switch (cfg.q_group_size) {
-            case 32: return launch_gemv_tma<1, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-            case 64: return launch_gemv_tma<2, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-            default: return launch_gemv_tma<4, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+            case 32: AWQ_GEMV_TMA(32);
+            case 64: AWQ_GEMV_TMA(64);
+            case 128: AWQ_GEMV_TMA(128);
+            default: AWQ_GEMV_TMA(256);
         }
+#undef AWQ_GEMV_TMA
     }
     switch (cfg.q_group_size) {
         case 32: return launch_gemv<1, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);

@@ -78,9 +78,12 @@ __host__ __device__ inline int gemv_ks(int units_per_row_group, int row_groups, 
     return ks;
 }
 
+// The MMA wrappers are not volatile: they are pure functions of their registers, and
+// leaving the compiler free to interleave independent accumulation chains hides the
+// MMA latency.
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -91,7 +94,7 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 __device__ __forceinline__ void mma_16816_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                 uint32_t b0, uint32_t b1) {
     const float z = 0.0f;
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%10, %10, %10, %10};"
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
@@ -338,7 +341,7 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
 // TMA-staged GEMV for N % 16 == 0 (every real layer): the same arithmetic as
 // gemv_mma_kernel with a different data path.
 //   * Weights reach shared memory through one 3-D tensor TMA copy per stage
-//     (16 rows x 2048 codes = 16 KB) issued by a producer warp into a 4-stage ring.
+//     (16 rows x 2048 codes = 16 KB) issued by a producer warp into a 5-stage ring.
 //     The 3-D view {16 words, rows, 128-code blocks} lands a stage as
 //     [block][row][64 B], so the two rows a quarter-warp reads are adjacent and the
 //     shared loads are conflict-free (row-major stages gave 8-way conflicts).
@@ -354,33 +357,44 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
 // ---------------------------------------------------------------------------
 
 constexpr int kTmaConsumers = 8;                            // consumer warps
-constexpr int kTmaThreads = (kTmaConsumers + 2) * 32;       // + producer warp + converter warp
-constexpr int kTmaStages = 4;
+constexpr int kTmaProducerWarp = kTmaConsumers;             // weight TMA copies
+constexpr int kTmaConverterWarp = kTmaConsumers + 1;        // scale/zero copies -> fp32 pairs
+constexpr int kTmaReducerWarp = kTmaConsumers + 2;          // partial sums -> Y
+constexpr int kTmaThreads = (kTmaConsumers + 3) * 32;
+constexpr int kTmaStages = 5;
+constexpr int kTmaParamSlots = 3;                           // row groups of parameters in flight
 constexpr int kTmaKC = 2048;                                // codes per row per stage
 constexpr int kTmaBlkBytes = kGemvRows * 64;               // one 128-code block of 16 rows
 constexpr int kTmaStageBytes = (kTmaKC / 128) * kTmaBlkBytes;
 
 struct GemvTmaSmem {
-    int K, M, nsteps, ng, nzw;
+    // K is padded to whole stages (Kp) in every shared-memory copy: X and its step sums
+    // are zero past K and so are the converted parameters past the last group, so the
+    // last, partial stage needs no validity checks.
+    int K, M, Kp, nsteps, nstepsp, ng, ngp, nzw;
     __host__ __device__ GemvTmaSmem(int M_, int K_, int G) : K(K_), M(M_) {
+        Kp = (K + kTmaKC - 1) / kTmaKC * kTmaKC;
         nsteps = K / (32 * gemv_words_per_thread(G));
+        nstepsp = Kp / (32 * gemv_words_per_thread(G));
         ng = K / G;
+        ngp = Kp / G;
         nzw = (ng + 7) / 8;
     }
     static __host__ __device__ size_t al16(size_t x) { return (x + 15) & ~(size_t)15; }
     __host__ __device__ size_t raw_scale_bytes() const { return (size_t)kGemvRows * ng * 2; }
     __host__ __device__ size_t raw_zero_bytes() const { return (size_t)kGemvRows * nzw * 4; }
     __host__ __device__ size_t raw_stride() const { return al16(raw_scale_bytes()) + al16(raw_zero_bytes()); }
-    __host__ __device__ size_t cvt_stride() const { return (size_t)kGemvRows * ng * 8; }
+    __host__ __device__ size_t cvt_stride() const { return (size_t)kGemvRows * ngp * 8; }
+    __host__ __device__ size_t part_stride() const { return (size_t)kTmaConsumers * kGemvRows * M * 4; }
     __host__ __device__ size_t raw() const { return (size_t)kTmaStages * kTmaStageBytes; }
-    __host__ __device__ size_t cvt() const { return raw() + 2 * raw_stride(); }
-    __host__ __device__ size_t x() const { return al16(cvt() + 2 * cvt_stride()); }
-    __host__ __device__ size_t xsum() const { return x() + (size_t)M * GemvSmem::x_pitch(K); }
-    __host__ __device__ size_t part() const { return al16(xsum() + (size_t)M * nsteps * 4); }
-    __host__ __device__ size_t zero() const { return part() + (size_t)2 * kTmaConsumers * kGemvRows * 8 * 4; }
+    __host__ __device__ size_t cvt() const { return raw() + kTmaParamSlots * raw_stride(); }
+    __host__ __device__ size_t x() const { return al16(cvt() + kTmaParamSlots * cvt_stride()); }
+    __host__ __device__ size_t xsum() const { return x() + (size_t)M * GemvSmem::x_pitch(Kp); }
+    __host__ __device__ size_t part() const { return al16(xsum() + (size_t)M * nstepsp * 4); }
+    __host__ __device__ size_t zero() const { return part() + 2 * part_stride(); }
     __host__ __device__ size_t bars() const { return (zero() + 64 + 7) & ~(size_t)7; }
-    // full[S], empty[S], pfull[2], rawfree[2], pready[2], pempty[2]
-    __host__ __device__ size_t bytes() const { return bars() + (2 * kTmaStages + 8) * 8; }
+    // full[S], empty[S], pfull/pready/pempty[PR], rfull/rempty[2]
+    __host__ __device__ size_t bytes() const { return bars() + (2 * kTmaStages + 3 * kTmaParamSlots + 4) * 8; }
 };
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -419,66 +433,63 @@ __device__ __forceinline__ void lds_words(uint32_t a, uint32_t* w) {
     }
 }
 
-template <int WT, bool ONE>
+// G is a template parameter so that every group index is a shift.  (FULL: K is a
+// multiple of kTmaKC; the padded layout makes both cases run the same loop.)
+template <int G, bool ONE, bool FULL>
 __global__ void __launch_bounds__(kTmaThreads, 2)
 gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __restrict__ X, int M,
-                const uint16_t* __restrict__ scales, const uint32_t* __restrict__ qzeros, int N, int K, int G,
+                const uint16_t* __restrict__ scales, const uint32_t* __restrict__ qzeros, int N, int K,
                 int zero_point, uint16_t* __restrict__ Y) {
     using namespace sm100;
+    constexpr int WT = gemv_words_per_thread(G);
     constexpr int kStepCodes = 32 * WT;
     constexpr int kStepsPerStage = kTmaKC / kStepCodes;
     constexpr int kStepsPerWarp = kStepsPerStage / kTmaConsumers;
+    constexpr int PR = kTmaParamSlots;
     extern __shared__ __align__(16) uint8_t smem[];
     const GemvTmaSmem L(M, K, G);
-    const int nsteps = L.nsteps, ng = L.ng, nzw = L.nzw;
+    const int ng = L.ng, ngp = L.ngp, nzw = L.nzw, nstepsp = L.nstepsp;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const bool zp = zero_point != 0;
     const int n_rg = N / kGemvRows;
     const int my_rg = blockIdx.x < n_rg ? (n_rg - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int nchunks = (K + kTmaKC - 1) / kTmaKC;
-    const int lg = 31 - __clz(G);
+    const int nchunks = L.Kp / kTmaKC;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars());
     uint64_t* empty = full + kTmaStages;
-    uint64_t* pfull = empty + kTmaStages;      // raw parameters landed
-    uint64_t* rawfree = pfull + 2;             // converter done with the raw buffer
-    uint64_t* pready = rawfree + 2;            // converted parameters ready
-    uint64_t* pempty = pready + 2;             // consumers done with the converted parameters
+    uint64_t* pfull = empty + kTmaStages;       // raw parameters landed
+    uint64_t* pready = pfull + PR;              // converted parameters ready
+    uint64_t* pempty = pready + PR;             // consumers done with converted parameters
+    uint64_t* rfull = pempty + PR;              // partial sums of a row group written
+    uint64_t* rempty = rfull + 2;               // reducer done with a partial-sum slot
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTmaStages; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], kTmaConsumers);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < PR; ++i) {
             mbar_init(&pfull[i], 1);
-            mbar_init(&rawfree[i], 1);
             mbar_init(&pready[i], 1);
             mbar_init(&pempty[i], kTmaConsumers);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&rfull[i], kTmaConsumers);
+            mbar_init(&rempty[i], 1);
         }
         mbar_fence_init();
         prefetch_tensormap(&tmap_q);
     }
     __syncthreads();
 
-    if (warp == kTmaConsumers) {
-        // ---------------- producer (weights, scales and zeros do not depend on X) ----------------
+    if (warp == kTmaProducerWarp) {
+        // ---------------- producer: the weight stream, gated only by free stages ----------------
         if (lane == 0) {
-            int stage = 0;
             bool ok = true;
-            const uint32_t pbytes = (uint32_t)(L.raw_scale_bytes() + (zp ? L.raw_zero_bytes() : 0));
+            int stage = 0;
             for (int rgi = 0; rgi < my_rg && ok; ++rgi) {
                 const int r0 = (blockIdx.x + rgi * gridDim.x) * kGemvRows;
-                const int pb = rgi & 1;
-                if (rgi >= 2) ok = mbar_wait(&rawfree[pb], ((rgi >> 1) - 1) & 1);
-                if (!ok) break;
-                uint8_t* raw = smem + L.raw() + pb * L.raw_stride();
-                mbar_arrive_expect_tx(&pfull[pb], pbytes);
-                bulk_g2s(raw, scales + (size_t)r0 * ng, (uint32_t)L.raw_scale_bytes(), &pfull[pb]);
-                if (zp)
-                    bulk_g2s(raw + L.al16(L.raw_scale_bytes()), qzeros + (size_t)r0 * nzw,
-                             (uint32_t)L.raw_zero_bytes(), &pfull[pb]);
-                for (int c = 0; c < nchunks && ok; ++c, ++stage) {
+                for (int c = 0; c < nchunks; ++c, ++stage) {
                     const int st = stage % kTmaStages;
                     if (stage >= kTmaStages && !(ok = mbar_wait(&empty[st], ((stage / kTmaStages) - 1) & 1))) break;
                     // box {16 words, 16 rows, 16 blocks}; blocks past K are filled with zeros
@@ -492,48 +503,107 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
         }
         return;
     }
-    if (warp == kTmaConsumers + 1) {
-        // ---------------- converter: raw scales/zeros -> (scale16 * 2^24, scale16 * zero) ----------------
+    if (warp == kTmaConverterWarp) {
+        // ---------------- converter: copies raw scales/zeros in, converts them to
+        // (scale16 * 2^24, scale16 * zero) pairs, PR row groups ahead of the consumers ----------------
+        const uint32_t pbytes = (uint32_t)(L.raw_scale_bytes() + (zp ? L.raw_zero_bytes() : 0));
+        auto issue_params = [&](int j) {
+            const int p = j % PR;
+            const int r0 = (blockIdx.x + j * gridDim.x) * kGemvRows;
+            uint8_t* raw = smem + L.raw() + p * L.raw_stride();
+            mbar_arrive_expect_tx(&pfull[p], pbytes);
+            bulk_g2s(raw, scales + (size_t)r0 * ng, (uint32_t)L.raw_scale_bytes(), &pfull[p]);
+            if (zp)
+                bulk_g2s(raw + L.al16(L.raw_scale_bytes()), qzeros + (size_t)r0 * nzw, (uint32_t)L.raw_zero_bytes(),
+                         &pfull[p]);
+        };
+        int issued = 0;
+        if (lane == 0)
+            for (int j = 0; j < PR && j < my_rg; ++j) issue_params(j);
+        issued = my_rg < PR ? my_rg : PR;
         bool ok = true;
-        for (int rgi = 0; rgi < my_rg && ok; ++rgi) {
-            const int pb = rgi & 1;
-            ok = mbar_wait(&pfull[pb], (rgi >> 1) & 1);
-            if (ok && rgi >= 2) ok = mbar_wait(&pempty[pb], ((rgi >> 1) - 1) & 1);
+        int rgi = 0;
+        for (; rgi < my_rg && ok; ++rgi) {
+            const int p = rgi % PR;
+            ok = mbar_wait(&pfull[p], (rgi / PR) & 1);
+            if (ok && rgi >= PR) ok = mbar_wait(&pempty[p], ((rgi / PR) - 1) & 1);
             if (!ok) break;
-            const uint8_t* raw = smem + L.raw() + pb * L.raw_stride();
+            const uint8_t* raw = smem + L.raw() + p * L.raw_stride();
             const uint16_t* rs = reinterpret_cast<const uint16_t*>(raw);
             const uint32_t* rz = reinterpret_cast<const uint32_t*>(raw + L.al16(L.raw_scale_bytes()));
-            float2* cv = reinterpret_cast<float2*>(smem + L.cvt() + pb * L.cvt_stride());
-            for (int e = lane; e < kGemvRows * ng; e += 32) {
-                const int r = e / ng, grp = e - r * ng;
-                const float sc = h2f(rs[e]);
-                const float z = zp ? (float)((rz[r * nzw + (grp >> 3)] >> (4 * (grp & 7))) & 15u) : 8.0f;
-                cv[e] = make_float2(sc * 16777216.0f, sc * z);
+            float2* cv = reinterpret_cast<float2*>(smem + L.cvt() + p * L.cvt_stride());
+            // lane = group within a run of 32; the 16 rows are independent and unrolled
+            for (int g0 = 0; g0 < ngp; g0 += 32) {
+                const int grp = g0 + lane;
+                if (grp < ngp) {
+                    const bool live = grp < ng;   // groups past K contribute nothing
+                    float sc[kGemvRows];
+                    uint32_t zw[kGemvRows];
+#pragma unroll
+                    for (int r = 0; r < kGemvRows; ++r) {
+                        sc[r] = live ? h2f(rs[r * ng + grp]) : 0.0f;
+                        zw[r] = (live && zp) ? rz[r * nzw + (grp >> 3)] : 0u;
+                    }
+                    const int sh = 4 * (grp & 7);
+#pragma unroll
+                    for (int r = 0; r < kGemvRows; ++r) {
+                        const float z = zp ? (float)((zw[r] >> sh) & 15u) : 8.0f;
+                        cv[r * ngp + grp] = make_float2(sc[r] * 16777216.0f, sc[r] * z);
+                    }
+                }
             }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&rawfree[pb]);
-                mbar_arrive(&pready[pb]);
+                mbar_arrive(&pready[p]);
+                // raw slot p has been read by the whole warp: refill it
+                if (rgi + PR < my_rg) issue_params(rgi + PR);
             }
+            if (rgi + PR < my_rg) ++issued;
+        }
+        // after a timeout, parameter copies still in flight must land before the CTA exits
+        if (lane == 0)
+            for (int j = issued - 1; j >= rgi && j >= issued - PR; --j) mbar_wait(&pfull[j % PR], (j / PR) & 1);
+        return;
+    }
+    if (warp == kTmaReducerWarp) {
+        // ---------------- reducer: add the 8 partial sums of each output in a fixed order ----------------
+        const float* part = reinterpret_cast<const float*>(smem + L.part());
+        for (int rgi = 0; rgi < my_rg; ++rgi) {
+            const int b = rgi & 1;
+            if (!mbar_wait(&rfull[b], (rgi >> 1) & 1)) break;
+            const float* slot = part + b * (L.part_stride() / 4);
+            const int n0 = (blockIdx.x + rgi * gridDim.x) * kGemvRows;
+            for (int o = lane; o < kGemvRows * M; o += 32) {
+                const int r = o / M, m = o - r * M;
+                float acc = 0.f;
+#pragma unroll
+                for (int w = 0; w < kTmaConsumers; ++w) acc += slot[w * kGemvRows * M + o];
+                Y[(size_t)m * N + n0 + r] = f2h_rn(acc);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rempty[b]);
         }
         return;
     }
 
-    // ---------------- consumers: stage X (permuted) and its per-step sums ----------------
+    // ---------------- consumers: stage X (permuted, zero past K) and its per-step sums ----------------
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const size_t pitch = GemvSmem::x_pitch(K);
+    const size_t pitch = GemvSmem::x_pitch(L.Kp);
     uint8_t* xs = smem + L.x();
     float* xsum = reinterpret_cast<float*>(smem + L.xsum());
-    const int kw = K >> 3;
+    const int kw = L.Kp >> 3;                 // words per padded row
+    const int kwv = K >> 3;                   // words per row that hold data
     constexpr int kCons = kTmaConsumers * 32;
     for (int u0 = threadIdx.x; u0 < M * kw; u0 += kCons * 4) {
         uint4 v[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int u = u0 + i * kCons;
+            v[i] = make_uint4(0, 0, 0, 0);
             if (u < M * kw) {
                 const int m = u / kw;
-                v[i] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)m * K + (u - m * kw) * 8));
+                const int word = u - m * kw;
+                if (word < kwv) v[i] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)m * K + word * 8));
             }
         }
 #pragma unroll
@@ -557,9 +627,9 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     if (threadIdx.x < 16) reinterpret_cast<uint32_t*>(smem + L.zero())[threadIdx.x] = 0u;
     asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    for (int u = threadIdx.x; u < M * nsteps; u += kCons) {
-        const int m = u / nsteps;
-        const int s = u - m * nsteps;
+    for (int u = threadIdx.x; u < M * nstepsp; u += kCons) {
+        const int m = u / nstepsp;
+        const int s = u - m * nstepsp;
         const uint4* xr = reinterpret_cast<const uint4*>(xs + m * pitch) + (size_t)s * WT * 4;
         float acc = 0.0f;
 #pragma unroll
@@ -574,94 +644,109 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
 
     // ---------------- consumers: stream the stages ----------------
+    // Every per-k-step shared address below is a per-stage base plus a compile-time
+    // offset.  Lanes whose B column is past M read X row 0: their D columns are never
+    // used, and a uniform stride keeps the offsets constant.
+    constexpr int Q = kStepsPerWarp;                 // k-steps of this warp per stage
+    constexpr int kStepsPerBlk = 4 / WT;             // k-steps per 128-code block
+    constexpr int R = G >= kStepCodes ? G / kStepCodes : 1;   // k-steps per group
     const int g = lane >> 2, t = lane & 3;
     const uint32_t sbase = smem_u32(smem);
-    // lane's B column: X row g, or the zero row when g >= M
-    const uint32_t xrow = g < M ? smem_u32(xs + g * pitch) + t * 16 : smem_u32(smem + L.zero()) + t * 16;
-    const uint32_t xstep = g < M ? 64u : 0u;
+    const uint32_t xrow = smem_u32(xs + (g < M ? g : 0) * pitch) + t * 16 + (uint32_t)(warp * Q * WT * 64);
     const int m0 = 2 * t, m1 = 2 * t + 1;
-    const uint32_t xs0 = smem_u32(xsum + (m0 < M ? m0 : 0) * nsteps);
-    const uint32_t xs1 = smem_u32(xsum + (m1 < M ? m1 : 0) * nsteps);
+    const uint32_t xs0 = smem_u32(xsum + (m0 < M ? m0 : 0) * nstepsp) + (uint32_t)(warp * Q * 4);
+    const uint32_t xs1 = smem_u32(xsum + (m1 < M ? m1 : 0) * nstepsp) + (uint32_t)(warp * Q * 4);
     const float xm0 = m0 < M ? 1.0f : 0.0f, xm1 = m1 < M ? 1.0f : 0.0f;
     const uint32_t cbase = smem_u32(smem + L.cvt());
     float* part = reinterpret_cast<float*>(smem + L.part());
-    // word w of row r in block b of a stage sits at b * kTmaBlkBytes + r * 64 + w * 4
-    const uint32_t wrow_a = (uint32_t)(g * 64 + t * WT * 4);
-    const uint32_t wrow_b = wrow_a + 8 * 64;
-    constexpr int kStepsPerBlk = 4 / WT;      // k-steps per 128-code block
-    const uint32_t prow_a = (uint32_t)(g * ng * 8), prow_b = (uint32_t)((g + 8) * ng * 8);
+    // weights: word w of row r in block b of a stage sits at b * kTmaBlkBytes + r * 64 + w * 4;
+    // this warp's first k-step of a stage starts a block (warp * Q is a multiple of kStepsPerBlk)
+    const uint32_t wrow = (uint32_t)((warp * Q / kStepsPerBlk) * kTmaBlkBytes + g * 64 + t * WT * 4);
+    const uint32_t prow_a = (uint32_t)(g * ngp * 8), prow_b = (uint32_t)((g + 8) * ngp * 8);
+    const int gwarp = (warp * Q) / R;                // group offset of the warp's first k-step in a stage
 
     int stage = 0;
     bool ok = true;
     for (int rgi = 0; rgi < my_rg; ++rgi) {
-        const int pb = rgi & 1;
-        ok = ok && mbar_wait(&pready[pb], (rgi >> 1) & 1);
-        const uint32_t cv = cbase + (uint32_t)(pb * L.cvt_stride());
+        const int p = rgi % PR;
+        ok = ok && mbar_wait(&pready[p], (rgi / PR) & 1);
+        const uint32_t cv = cbase + (uint32_t)(p * L.cvt_stride());
+        const uint32_t cva = cv + prow_a + (uint32_t)(gwarp * 8), cvb = cv + prow_b + (uint32_t)(gwarp * 8);
         float y[4] = {0.f, 0.f, 0.f, 0.f};
         for (int c = 0; c < nchunks; ++c, ++stage) {
             const int st = stage % kTmaStages;
             ok = ok && mbar_wait(&full[st], (stage / kTmaStages) & 1);
-            const uint32_t sb = sbase + (uint32_t)(st * kTmaStageBytes);
+            const uint32_t sb = sbase + (uint32_t)(st * kTmaStageBytes) + wrow;
+            const uint32_t xb = xrow + (uint32_t)(c * kStepsPerStage * WT * 64);
+            const uint32_t gb = (uint32_t)(c * (kStepsPerStage / R) * 8);
+            const uint32_t x0b = xs0 + (uint32_t)(c * kStepsPerStage * 4);
+            const uint32_t x1b = xs1 + (uint32_t)(c * kStepsPerStage * 4);
+            // the warp's Q k-steps as straight-line code: fragment loads, then independent
+            // MMA chains interleaved, then the folds
+            uint32_t wa[Q][WT], wb[Q][WT];
 #pragma unroll
-            for (int q = 0; q < kStepsPerWarp; ++q) {
-                const int ks = warp * kStepsPerWarp + q;          // k-step inside the stage
-                const int s = c * kStepsPerStage + ks;            // k-step inside the row
-                if (!ok || s >= nsteps) break;
-                uint32_t wa[WT], wb[WT];
-                const uint32_t koff = (uint32_t)((ks / kStepsPerBlk) * kTmaBlkBytes + (ks % kStepsPerBlk) * WT * 16);
-                lds_words<WT>(sb + wrow_a + koff, wa);
-                lds_words<WT>(sb + wrow_b + koff, wb);
-                float d1[4], d16[4];
+            for (int q = 0; q < Q; ++q) {
+                const uint32_t off = (uint32_t)((q / kStepsPerBlk) * kTmaBlkBytes + (q % kStepsPerBlk) * WT * 16);
+                lds_words<WT>(sb + off, wa[q]);
+                lds_words<WT>(sb + off + 8 * 64, wb[q]);
+            }
+            float d1[Q][4], d16[Q][4];
 #pragma unroll
-                for (int j = 0; j < WT; ++j) {
-                    const uint4 b = lds128(xrow + (uint32_t)(s * WT + j) * xstep);
-                    const uint32_t wa8 = wa[j] >> 8, wb8 = wb[j] >> 8;
+            for (int j = 0; j < WT; ++j) {
+#pragma unroll
+                for (int q = 0; q < Q; ++q) {
+                    const uint4 b = lds128(xb + (uint32_t)((q * WT + j) * 64));
+                    const uint32_t a = wa[q][j], bb = wb[q][j];
+                    const uint32_t a8 = a >> 8, b8 = bb >> 8;
                     if (j == 0) {
-                        mma_16816_first(d1, wa[j] & 0x000F000Fu, wb[j] & 0x000F000Fu, wa8 & 0x000F000Fu,
-                                        wb8 & 0x000F000Fu, b.x, b.y);
-                        mma_16816_first(d16, wa[j] & 0x00F000F0u, wb[j] & 0x00F000F0u, wa8 & 0x00F000F0u,
-                                        wb8 & 0x00F000F0u, b.z, b.w);
+                        mma_16816_first(d1[q], a & 0x000F000Fu, bb & 0x000F000Fu, a8 & 0x000F000Fu,
+                                        b8 & 0x000F000Fu, b.x, b.y);
+                        mma_16816_first(d16[q], a & 0x00F000F0u, bb & 0x00F000F0u, a8 & 0x00F000F0u,
+                                        b8 & 0x00F000F0u, b.z, b.w);
                     } else {
-                        mma_16816(d1, wa[j] & 0x000F000Fu, wb[j] & 0x000F000Fu, wa8 & 0x000F000Fu,
-                                  wb8 & 0x000F000Fu, b.x, b.y);
-                        mma_16816(d16, wa[j] & 0x00F000F0u, wb[j] & 0x00F000F0u, wa8 & 0x00F000F0u,
-                                  wb8 & 0x00F000F0u, b.z, b.w);
+                        mma_16816(d1[q], a & 0x000F000Fu, bb & 0x000F000Fu, a8 & 0x000F000Fu, b8 & 0x000F000Fu,
+                                  b.x, b.y);
+                        mma_16816(d16[q], a & 0x00F000F0u, bb & 0x00F000F0u, a8 & 0x00F000F0u,
+                                  b8 & 0x00F000F0u, b.z, b.w);
                     }
                 }
+            }
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
                 // fold: y += (scale16 2^24) (D1 + D16/16) - (scale16 z) sum_k x
-                const int grp = (s * kStepCodes) >> lg;
-                const uint2 pa = lds64(cv + prow_a + grp * 8);
-                const uint2 pbv = lds64(cv + prow_b + grp * 8);
-                const float x0 = ldsf(xs0 + s * 4) * xm0;
-                y[0] = fmaf(__uint_as_float(pa.x), fmaf(d16[0], 0.0625f, d1[0]), fmaf(-__uint_as_float(pa.y), x0, y[0]));
-                y[2] = fmaf(__uint_as_float(pbv.x), fmaf(d16[2], 0.0625f, d1[2]), fmaf(-__uint_as_float(pbv.y), x0, y[2]));
+                const uint32_t go = gb + (uint32_t)((q / R) * 8);
+                const uint2 pa = lds64(cva + go);
+                const uint2 pbv = lds64(cvb + go);
+                const float x0 = ldsf(x0b + (uint32_t)(q * 4)) * xm0;
+                const float sa = __uint_as_float(pa.x), sza = __uint_as_float(pa.y);
+                const float sb2 = __uint_as_float(pbv.x), szb = __uint_as_float(pbv.y);
+                y[0] = fmaf(sa, fmaf(d16[q][0], 0.0625f, d1[q][0]), fmaf(-sza, x0, y[0]));
+                y[2] = fmaf(sb2, fmaf(d16[q][2], 0.0625f, d1[q][2]), fmaf(-szb, x0, y[2]));
                 if (!ONE) {
-                    const float x1 = ldsf(xs1 + s * 4) * xm1;
-                    y[1] = fmaf(__uint_as_float(pa.x), fmaf(d16[1], 0.0625f, d1[1]), fmaf(-__uint_as_float(pa.y), x1, y[1]));
-                    y[3] = fmaf(__uint_as_float(pbv.x), fmaf(d16[3], 0.0625f, d1[3]), fmaf(-__uint_as_float(pbv.y), x1, y[3]));
+                    const float x1 = ldsf(x1b + (uint32_t)(q * 4)) * xm1;
+                    y[1] = fmaf(sa, fmaf(d16[q][1], 0.0625f, d1[q][1]), fmaf(-sza, x1, y[1]));
+                    y[3] = fmaf(sb2, fmaf(d16[q][3], 0.0625f, d1[q][3]), fmaf(-szb, x1, y[3]));
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
         }
-        // row group done: parameters released; combine the 8 partial sums in a fixed order
         __syncwarp();
-        if (lane == 0) mbar_arrive(&pempty[pb]);
-        float* slot = part + pb * (kTmaConsumers * kGemvRows * 8);
-        float* pw = slot + warp * kGemvRows * 8;
-        pw[g * 8 + 2 * t] = y[0];
-        pw[g * 8 + 2 * t + 1] = y[1];
-        pw[(g + 8) * 8 + 2 * t] = y[2];
-        pw[(g + 8) * 8 + 2 * t + 1] = y[3];
-        asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
-        if (threadIdx.x < kGemvRows * 8) {
-            const int r = threadIdx.x >> 3, m = threadIdx.x & 7;
-            float acc = 0.f;
-#pragma unroll
-            for (int w = 0; w < kTmaConsumers; ++w) acc += slot[w * kGemvRows * 8 + threadIdx.x];
-            const int n = (blockIdx.x + rgi * gridDim.x) * kGemvRows + r;
-            if (m < M) Y[(size_t)m * N + n] = f2h_rn(acc);
+        if (lane == 0) mbar_arrive(&pempty[p]);
+        // hand the partial sums to the reducer warp (no CTA-wide barrier)
+        const int b = rgi & 1;
+        if (rgi >= 2) ok = ok && mbar_wait(&rempty[b], ((rgi >> 1) - 1) & 1);
+        float* pw = part + b * (L.part_stride() / 4) + warp * kGemvRows * M;
+        if (m0 < M) {
+            pw[g * M + m0] = y[0];
+            pw[(g + 8) * M + m0] = y[2];
         }
+        if (m1 < M) {
+            pw[g * M + m1] = y[1];
+            pw[(g + 8) * M + m1] = y[3];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rfull[b]);
     }
 }
 
