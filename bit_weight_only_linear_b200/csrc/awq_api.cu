@@ -23,6 +23,7 @@ struct DeviceInfo {
     bool ready = false;
     int sms = 0;
     int max_smem_optin = 0;
+    int smem_per_sm = 0;
 };
 
 std::mutex g_mu;
@@ -37,6 +38,8 @@ bool device_info(DeviceInfo& out) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
         if (cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
             cudaSuccess)
+            return false;
+        if (cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
             return false;
         d.ready = true;
     }
@@ -122,30 +125,42 @@ awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const 
     return launch_status();
 }
 
-template <int G, bool ONE, bool FULL>
+// Stages and raw parameter slots of the TMA GEMV: the deepest ring (3..6 stages) with
+// which two CTAs fit on an SM, else the deepest with which one fits; false if none fits.
+bool pick_gemv_tma(const DeviceInfo& d, int M, int K, int G, int& S, int& PR) {
+    PR = GemvTmaSmem::param_slots(K);
+    for (int ctas = 2; ctas >= 1; --ctas)
+        for (S = kTmaMaxStages; S >= kTmaMinStages; --S) {
+            const size_t b = GemvTmaSmem(M, K, G, S, PR).bytes();
+            if (b <= (size_t)d.max_smem_optin && (size_t)ctas * (b + 1024) <= (size_t)d.smem_per_sm) return true;
+        }
+    return false;
+}
+
+template <int G, bool ONE>
 awq_status launch_gemv_tma(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
                            const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
                            cudaStream_t st) {
     DeviceInfo d;
     if (!device_info(d)) return AWQ_ERR_CUDA;
-    const GemvTmaSmem L(M, K, cfg.q_group_size);
-    const size_t smem = L.bytes();
+    int S = 0, PR = 0;
+    if (!pick_gemv_tma(d, M, K, G, S, PR)) return AWQ_ERR_UNSUPPORTED;
+    const size_t smem = GemvTmaSmem(M, K, G, S, PR).bytes();
     // qweight [N][K/8] words viewed as {16 words, N rows, K/128 blocks}
     CUtensorMap tq;
     if (!make_tmap_3d(&tq, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 16, (uint64_t)N, (uint64_t)(K / 128),
                       (uint64_t)K / 2, 64, 16, kGemvRows, kTmaKC / 128))
         return AWQ_ERR_CUDA;
-    if (smem > (size_t)d.max_smem_optin) return AWQ_ERR_UNSUPPORTED;
-    auto kern = gemv_tma_kernel<G, ONE, FULL>;
+    auto kern = gemv_tma_kernel<G, ONE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return AWQ_ERR_CUDA;
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kTmaThreads, smem) != cudaSuccess || occ < 1)
         return AWQ_ERR_CUDA;
+    // one CTA per resident slot, row groups dealt round-robin
     const int n_rg = N / kGemvRows;
     const int slots = d.sms * occ;
-    const int per_cta = ceil_div(n_rg, slots);
-    const int grid = ceil_div(n_rg, per_cta);
+    const int grid = n_rg < slots ? n_rg : slots;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(grid);
     lc.blockDim = dim3(kTmaThreads);
@@ -156,7 +171,8 @@ awq_status launch_gemv_tma(const uint16_t* X, int M, const uint32_t* qweight, co
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&lc, kern, tq, X, M, scales, qzeros, N, K, (int)cfg.zero_point, Y) != cudaSuccess)
+    if (cudaLaunchKernelEx(&lc, kern, tq, X, M, scales, qzeros, N, K, (int)cfg.zero_point, Y, S, PR) !=
+        cudaSuccess)
         return AWQ_ERR_CUDA;
     return launch_status();
 }
@@ -170,19 +186,18 @@ awq_status dispatch_gemv(const uint16_t* X, int M, const uint32_t* qweight, cons
     DeviceInfo d;
     if (!device_info(d)) return AWQ_ERR_CUDA;
     if (N % kGemvRows == 0 && K % 128 == 0 && (uintptr_t)scales % 16 == 0 &&
-        (!cfg.zero_point || (uintptr_t)qzeros % 16 == 0) &&
-        GemvTmaSmem(M, K, cfg.q_group_size).bytes() <= (size_t)d.max_smem_optin) {
-        const bool full = K % kTmaKC == 0;
-#define AWQ_GEMV_TMA(GG)                                                                                   \
-    return full ? launch_gemv_tma<GG, ONE, true>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s)          \
-                : launch_gemv_tma<GG, ONE, false>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s)
-        switch (cfg.q_group_size) {
-            case 32: AWQ_GEMV_TMA(32);
-            case 64: AWQ_GEMV_TMA(64);
-            case 128: AWQ_GEMV_TMA(128);
-            default: AWQ_GEMV_TMA(256);
-        }
+        (!cfg.zero_point || (uintptr_t)qzeros % 16 == 0)) {
+        int S = 0, PR = 0;
+        if (pick_gemv_tma(d, M, K, cfg.q_group_size, S, PR)) {
+#define AWQ_GEMV_TMA(GG) return launch_gemv_tma<GG, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s)
+            switch (cfg.q_group_size) {
+                case 32: AWQ_GEMV_TMA(32);
+                case 64: AWQ_GEMV_TMA(64);
+                case 128: AWQ_GEMV_TMA(128);
+                default: AWQ_GEMV_TMA(256);
+            }
 #undef AWQ_GEMV_TMA
+        }
     }
     switch (cfg.q_group_size) {
         case 32: return launch_gemv<1, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);

@@ -341,19 +341,23 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
 // TMA-staged GEMV for N % 16 == 0 (every real layer): the same arithmetic as
 // gemv_mma_kernel with a different data path.
 //   * Weights reach shared memory through one 3-D tensor TMA copy per stage
-//     (16 rows x 2048 codes = 16 KB) issued by a producer warp into a 5-stage ring.
-//     The 3-D view {16 words, rows, 128-code blocks} lands a stage as
+//     (16 rows x 2048 codes = 16 KB) issued by a producer warp into a ring of S
+//     stages.  The 3-D view {16 words, rows, 128-code blocks} lands a stage as
 //     [block][row][64 B], so the two rows a quarter-warp reads are adjacent and the
 //     shared loads are conflict-free (row-major stages gave 8-way conflicts).
 //     Measured on B200: 16 per-row bulk copies per stage cap the copy rate near
-//     2 TB/s; one tensor copy per stage does not.
-//   * Scales and zero words of a row group arrive through two bulk copies into a raw
-//     parameter buffer; a converter warp turns them into fp32 pairs
-//     (scale16 * 2^24, scale16 * zero) per (row, group), so the consumers' fold is
-//     two shared loads and three FMAs per row.
+//     2 TB/s; one tensor copy per stage does not.  The producer waits for nothing
+//     but a free stage.
+//   * Scales and zero words of a row group arrive through two bulk copies into a
+//     ring of PR raw parameter slots.  A converter warp turns the groups of each
+//     stage into fp32 pairs (scale16 * 2^24, scale16 * zero) in a small buffer that
+//     belongs to the stage: a stage is full when both its TMA bytes and the
+//     converter's arrival are in, and both refill it after the consumers release
+//     it.  Per-stage buffers keep the footprint of long rows small enough for two
+//     CTAs per SM.
 //   * The 8 consumer warps run only the decode, the MMAs and the fold, each taking
-//     1/8 of a stage's k-steps; no register ring, no global address math, no
-//     predication.  Every wait is bounded.
+//     1/8 of a stage's k-steps; a reducer warp adds their partial sums in a fixed
+//     order.  Every wait is bounded.
 // ---------------------------------------------------------------------------
 
 constexpr int kTmaConsumers = 8;                            // consumer warps
@@ -361,8 +365,7 @@ constexpr int kTmaProducerWarp = kTmaConsumers;             // weight TMA copies
 constexpr int kTmaConverterWarp = kTmaConsumers + 1;        // scale/zero copies -> fp32 pairs
 constexpr int kTmaReducerWarp = kTmaConsumers + 2;          // partial sums -> Y
 constexpr int kTmaThreads = (kTmaConsumers + 3) * 32;
-constexpr int kTmaStages = 5;
-constexpr int kTmaParamSlots = 3;                           // row groups of parameters in flight
+constexpr int kTmaMinStages = 3, kTmaMaxStages = 6;
 constexpr int kTmaKC = 2048;                                // codes per row per stage
 constexpr int kTmaBlkBytes = kGemvRows * 64;               // one 128-code block of 16 rows
 constexpr int kTmaStageBytes = (kTmaKC / 128) * kTmaBlkBytes;
@@ -371,30 +374,33 @@ struct GemvTmaSmem {
     // K is padded to whole stages (Kp) in every shared-memory copy: X and its step sums
     // are zero past K and so are the converted parameters past the last group, so the
     // last, partial stage needs no validity checks.
-    int K, M, Kp, nsteps, nstepsp, ng, ngp, nzw;
-    __host__ __device__ GemvTmaSmem(int M_, int K_, int G) : K(K_), M(M_) {
+    int K, M, S, PR, Kp, nstepsp, ng, nzw, gpc;
+    __host__ __device__ GemvTmaSmem(int M_, int K_, int G, int S_, int PR_) : K(K_), M(M_), S(S_), PR(PR_) {
         Kp = (K + kTmaKC - 1) / kTmaKC * kTmaKC;
-        nsteps = K / (32 * gemv_words_per_thread(G));
         nstepsp = Kp / (32 * gemv_words_per_thread(G));
         ng = K / G;
-        ngp = Kp / G;
         nzw = (ng + 7) / 8;
+        gpc = kTmaKC / G;
+    }
+    // raw parameter slots for a row group: PR = 4, 3, 2 for 1, 2-3, >= 4 stages per row
+    static __host__ __device__ int param_slots(int K) {
+        const int nchunks = (K + kTmaKC - 1) / kTmaKC;
+        return nchunks >= 4 ? 2 : (nchunks >= 2 ? 3 : 4);
     }
     static __host__ __device__ size_t al16(size_t x) { return (x + 15) & ~(size_t)15; }
     __host__ __device__ size_t raw_scale_bytes() const { return (size_t)kGemvRows * ng * 2; }
     __host__ __device__ size_t raw_zero_bytes() const { return (size_t)kGemvRows * nzw * 4; }
     __host__ __device__ size_t raw_stride() const { return al16(raw_scale_bytes()) + al16(raw_zero_bytes()); }
-    __host__ __device__ size_t cvt_stride() const { return (size_t)kGemvRows * ngp * 8; }
+    __host__ __device__ size_t cvt_stride() const { return (size_t)kGemvRows * gpc * 8; }
     __host__ __device__ size_t part_stride() const { return (size_t)kTmaConsumers * kGemvRows * M * 4; }
-    __host__ __device__ size_t raw() const { return (size_t)kTmaStages * kTmaStageBytes; }
-    __host__ __device__ size_t cvt() const { return raw() + kTmaParamSlots * raw_stride(); }
-    __host__ __device__ size_t x() const { return al16(cvt() + kTmaParamSlots * cvt_stride()); }
+    __host__ __device__ size_t raw() const { return (size_t)S * kTmaStageBytes; }
+    __host__ __device__ size_t cvt() const { return raw() + PR * raw_stride(); }
+    __host__ __device__ size_t x() const { return al16(cvt() + S * cvt_stride()); }
     __host__ __device__ size_t xsum() const { return x() + (size_t)M * GemvSmem::x_pitch(Kp); }
     __host__ __device__ size_t part() const { return al16(xsum() + (size_t)M * nstepsp * 4); }
-    __host__ __device__ size_t zero() const { return part() + 2 * part_stride(); }
-    __host__ __device__ size_t bars() const { return (zero() + 64 + 7) & ~(size_t)7; }
-    // full[S], empty[S], pfull/pready/pempty[PR], rfull/rempty[2]
-    __host__ __device__ size_t bytes() const { return bars() + (2 * kTmaStages + 3 * kTmaParamSlots + 4) * 8; }
+    __host__ __device__ size_t bars() const { return (part() + 2 * part_stride() + 7) & ~(size_t)7; }
+    // full[S], empty[S], pfull[PR], rfull[2], rempty[2]
+    __host__ __device__ size_t bytes() const { return bars() + (2 * S + PR + 4) * 8; }
 };
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -433,46 +439,40 @@ __device__ __forceinline__ void lds_words(uint32_t a, uint32_t* w) {
     }
 }
 
-// G is a template parameter so that every group index is a shift.  (FULL: K is a
-// multiple of kTmaKC; the padded layout makes both cases run the same loop.)
-template <int G, bool ONE, bool FULL>
+// G is a template parameter so that every group index is a shift.  S (stages) and
+// PR (raw parameter slots) are chosen by the host from the shared-memory budget.
+template <int G, bool ONE>
 __global__ void __launch_bounds__(kTmaThreads, 2)
 gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __restrict__ X, int M,
                 const uint16_t* __restrict__ scales, const uint32_t* __restrict__ qzeros, int N, int K,
-                int zero_point, uint16_t* __restrict__ Y) {
+                int zero_point, uint16_t* __restrict__ Y, int S, int PR) {
     using namespace sm100;
     constexpr int WT = gemv_words_per_thread(G);
     constexpr int kStepCodes = 32 * WT;
     constexpr int kStepsPerStage = kTmaKC / kStepCodes;
-    constexpr int kStepsPerWarp = kStepsPerStage / kTmaConsumers;
-    constexpr int PR = kTmaParamSlots;
+    constexpr int Q = kStepsPerStage / kTmaConsumers;           // k-steps of a warp per stage
+    constexpr int GPC = kTmaKC / G;                             // groups per stage
     extern __shared__ __align__(16) uint8_t smem[];
-    const GemvTmaSmem L(M, K, G);
-    const int ng = L.ng, ngp = L.ngp, nzw = L.nzw, nstepsp = L.nstepsp;
+    const GemvTmaSmem L(M, K, G, S, PR);
+    const int ng = L.ng, nzw = L.nzw, nstepsp = L.nstepsp;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const bool zp = zero_point != 0;
     const int n_rg = N / kGemvRows;
     const int my_rg = blockIdx.x < n_rg ? (n_rg - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const int nchunks = L.Kp / kTmaKC;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars());
-    uint64_t* empty = full + kTmaStages;
-    uint64_t* pfull = empty + kTmaStages;       // raw parameters landed
-    uint64_t* pready = pfull + PR;              // converted parameters ready
-    uint64_t* pempty = pready + PR;             // consumers done with converted parameters
-    uint64_t* rfull = pempty + PR;              // partial sums of a row group written
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars());   // weights + converted params in
+    uint64_t* empty = full + S;                 // consumers done with a stage
+    uint64_t* pfull = empty + S;                // raw parameters of a row group landed
+    uint64_t* rfull = pfull + PR;               // partial sums of a row group written
     uint64_t* rempty = rfull + 2;               // reducer done with a partial-sum slot
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kTmaStages; ++i) {
-            mbar_init(&full[i], 1);
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 2);             // producer (with its bytes) + converter
             mbar_init(&empty[i], kTmaConsumers);
         }
-        for (int i = 0; i < PR; ++i) {
-            mbar_init(&pfull[i], 1);
-            mbar_init(&pready[i], 1);
-            mbar_init(&pempty[i], kTmaConsumers);
-        }
+        for (int i = 0; i < PR; ++i) mbar_init(&pfull[i], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&rfull[i], kTmaConsumers);
             mbar_init(&rempty[i], 1);
@@ -486,26 +486,27 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
         // ---------------- producer: the weight stream, gated only by free stages ----------------
         if (lane == 0) {
             bool ok = true;
-            int stage = 0;
+            int stage = 0, st = 0;
+            uint32_t ph = 0;                    // parity of the current use of slot st
             for (int rgi = 0; rgi < my_rg && ok; ++rgi) {
                 const int r0 = (blockIdx.x + rgi * gridDim.x) * kGemvRows;
-                for (int c = 0; c < nchunks; ++c, ++stage) {
-                    const int st = stage % kTmaStages;
-                    if (stage >= kTmaStages && !(ok = mbar_wait(&empty[st], ((stage / kTmaStages) - 1) & 1))) break;
+                for (int c = 0; c < nchunks; ++c) {
+                    if (stage >= S && !(ok = mbar_wait(&empty[st], ph ^ 1u))) break;
                     // box {16 words, 16 rows, 16 blocks}; blocks past K are filled with zeros
                     mbar_arrive_expect_tx(&full[st], kTmaStageBytes);
                     tma_load_3d(smem + (size_t)st * kTmaStageBytes, &tmap_q, &full[st], 0, r0, c * (kTmaKC / 128));
+                    ++stage;
+                    if (++st == S) { st = 0; ph ^= 1u; }
                 }
             }
             // drain: copies in flight must land before the CTA exits
-            for (int s2 = stage - 1; s2 >= 0 && s2 >= stage - kTmaStages; --s2)
-                mbar_wait(&full[s2 % kTmaStages], (s2 / kTmaStages) & 1);
+            for (int s2 = stage - 1; s2 >= 0 && s2 >= stage - S; --s2) mbar_wait(&full[s2 % S], (s2 / S) & 1);
         }
         return;
     }
     if (warp == kTmaConverterWarp) {
-        // ---------------- converter: copies raw scales/zeros in, converts them to
-        // (scale16 * 2^24, scale16 * zero) pairs, PR row groups ahead of the consumers ----------------
+        // ---------------- converter: raw scales/zeros of a row group -> per-stage
+        // (scale16 * 2^24, scale16 * zero) pairs ----------------
         const uint32_t pbytes = (uint32_t)(L.raw_scale_bytes() + (zp ? L.raw_zero_bytes() : 0));
         auto issue_params = [&](int j) {
             const int p = j % PR;
@@ -517,47 +518,50 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
                 bulk_g2s(raw + L.al16(L.raw_scale_bytes()), qzeros + (size_t)r0 * nzw, (uint32_t)L.raw_zero_bytes(),
                          &pfull[p]);
         };
-        int issued = 0;
         if (lane == 0)
             for (int j = 0; j < PR && j < my_rg; ++j) issue_params(j);
-        issued = my_rg < PR ? my_rg : PR;
+        int issued = my_rg < PR ? my_rg : PR;
         bool ok = true;
-        int rgi = 0;
+        int rgi = 0, stage = 0, st = 0;
+        uint32_t ph = 0;
+        constexpr int EPL = kGemvRows * GPC / 32;             // (row, group) pairs per lane per stage
+        constexpr int EB = EPL < 8 ? EPL : 8;                 // converted in batches of EB
         for (; rgi < my_rg && ok; ++rgi) {
             const int p = rgi % PR;
-            ok = mbar_wait(&pfull[p], (rgi / PR) & 1);
-            if (ok && rgi >= PR) ok = mbar_wait(&pempty[p], ((rgi / PR) - 1) & 1);
-            if (!ok) break;
+            if (!(ok = mbar_wait(&pfull[p], (rgi / PR) & 1))) break;
             const uint8_t* raw = smem + L.raw() + p * L.raw_stride();
             const uint16_t* rs = reinterpret_cast<const uint16_t*>(raw);
             const uint32_t* rz = reinterpret_cast<const uint32_t*>(raw + L.al16(L.raw_scale_bytes()));
-            float2* cv = reinterpret_cast<float2*>(smem + L.cvt() + p * L.cvt_stride());
-            // lane = group within a run of 32; the 16 rows are independent and unrolled
-            for (int g0 = 0; g0 < ngp; g0 += 32) {
-                const int grp = g0 + lane;
-                if (grp < ngp) {
-                    const bool live = grp < ng;   // groups past K contribute nothing
-                    float sc[kGemvRows];
-                    uint32_t zw[kGemvRows];
+            for (int c = 0; c < nchunks; ++c) {
+                if (stage >= S && !(ok = mbar_wait(&empty[st], ph ^ 1u))) break;
+                float2* cv = reinterpret_cast<float2*>(smem + L.cvt() + (size_t)st * L.cvt_stride());
+                for (int i0 = 0; i0 < EPL; i0 += EB) {
+                    float sc[EB];
+                    uint32_t zw[EB];
 #pragma unroll
-                    for (int r = 0; r < kGemvRows; ++r) {
-                        sc[r] = live ? h2f(rs[r * ng + grp]) : 0.0f;
-                        zw[r] = (live && zp) ? rz[r * nzw + (grp >> 3)] : 0u;
+                    for (int i = 0; i < EB; ++i) {
+                        const int e = lane + 32 * (i0 + i);
+                        const int r = e / GPC, grp = c * GPC + (e % GPC);
+                        const bool live = grp < ng;   // groups past K contribute nothing
+                        sc[i] = live ? h2f(rs[r * ng + grp]) : 0.0f;
+                        zw[i] = (live && zp) ? rz[r * nzw + (grp >> 3)] : 0u;
                     }
-                    const int sh = 4 * (grp & 7);
 #pragma unroll
-                    for (int r = 0; r < kGemvRows; ++r) {
-                        const float z = zp ? (float)((zw[r] >> sh) & 15u) : 8.0f;
-                        cv[r * ngp + grp] = make_float2(sc[r] * 16777216.0f, sc[r] * z);
+                    for (int i = 0; i < EB; ++i) {
+                        const int e = lane + 32 * (i0 + i);
+                        const int grp = c * GPC + (e % GPC);
+                        const float z = zp ? (float)((zw[i] >> (4 * (grp & 7))) & 15u) : 8.0f;
+                        cv[e] = make_float2(sc[i] * 16777216.0f, sc[i] * z);
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[st]);
+                ++stage;
+                if (++st == S) { st = 0; ph ^= 1u; }
             }
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&pready[p]);
-                // raw slot p has been read by the whole warp: refill it
-                if (rgi + PR < my_rg) issue_params(rgi + PR);
-            }
+            if (!ok) break;
+            // the whole warp has read raw slot p: refill it
+            if (lane == 0 && rgi + PR < my_rg) issue_params(rgi + PR);
             if (rgi + PR < my_rg) ++issued;
         }
         // after a timeout, parameter copies still in flight must land before the CTA exits
@@ -624,22 +628,33 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
             }
         }
     }
-    if (threadIdx.x < 16) reinterpret_cast<uint32_t*>(smem + L.zero())[threadIdx.x] = 0u;
     asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    for (int u = threadIdx.x; u < M * nstepsp; u += kCons) {
-        const int m = u / nstepsp;
-        const int s = u - m * nstepsp;
-        const uint4* xr = reinterpret_cast<const uint4*>(xs + m * pitch) + (size_t)s * WT * 4;
-        float acc = 0.0f;
+    {
+        // TPS threads per (row, k-step), each adding UPT 16-byte chunks, then a
+        // butterfly over the TPS lanes
+        constexpr int TPS = 4 * WT < 8 ? 4 * WT : 8;
+        constexpr int UPT = 4 * WT / TPS;
+        const int items = M * nstepsp * TPS;
+        for (int u0 = 0; u0 < items; u0 += kCons) {
+            const int u = u0 + threadIdx.x;
+            float acc = 0.0f;
+            if (u < items) {
+                const int ms = u / TPS, part = u % TPS;
+                const int m = ms / nstepsp, s = ms - m * nstepsp;
+                const uint4* xr = reinterpret_cast<const uint4*>(xs + m * pitch) + (size_t)s * WT * 4 + part * UPT;
 #pragma unroll
-        for (int i = 0; i < 4 * WT; ++i) {
-            const uint4 v = xr[i];
-            const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
+                for (int i = 0; i < UPT; ++i) {
+                    const uint4 v = xr[i];
+                    const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc += h2f(h[e]);
+                    for (int e = 0; e < 8; ++e) acc += h2f(h[e]);
+                }
+            }
+#pragma unroll
+            for (int o = TPS / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (u < items && u % TPS == 0) xsum[u / TPS] = acc;
         }
-        xsum[u] = acc;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
 
@@ -647,7 +662,6 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     // Every per-k-step shared address below is a per-stage base plus a compile-time
     // offset.  Lanes whose B column is past M read X row 0: their D columns are never
     // used, and a uniform stride keeps the offsets constant.
-    constexpr int Q = kStepsPerWarp;                 // k-steps of this warp per stage
     constexpr int kStepsPerBlk = 4 / WT;             // k-steps per 128-code block
     constexpr int R = G >= kStepCodes ? G / kStepCodes : 1;   // k-steps per group
     const int g = lane >> 2, t = lane & 3;
@@ -657,28 +671,24 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     const uint32_t xs0 = smem_u32(xsum + (m0 < M ? m0 : 0) * nstepsp) + (uint32_t)(warp * Q * 4);
     const uint32_t xs1 = smem_u32(xsum + (m1 < M ? m1 : 0) * nstepsp) + (uint32_t)(warp * Q * 4);
     const float xm0 = m0 < M ? 1.0f : 0.0f, xm1 = m1 < M ? 1.0f : 0.0f;
-    const uint32_t cbase = smem_u32(smem + L.cvt());
     float* part = reinterpret_cast<float*>(smem + L.part());
     // weights: word w of row r in block b of a stage sits at b * kTmaBlkBytes + r * 64 + w * 4;
     // this warp's first k-step of a stage starts a block (warp * Q is a multiple of kStepsPerBlk)
     const uint32_t wrow = (uint32_t)((warp * Q / kStepsPerBlk) * kTmaBlkBytes + g * 64 + t * WT * 4);
-    const uint32_t prow_a = (uint32_t)(g * ngp * 8), prow_b = (uint32_t)((g + 8) * ngp * 8);
-    const int gwarp = (warp * Q) / R;                // group offset of the warp's first k-step in a stage
+    // converted parameters of a stage: [row][group of the stage] fp32 pairs
+    const uint32_t prow = smem_u32(smem + L.cvt()) + (uint32_t)(g * GPC * 8 + ((warp * Q) / R) * 8);
+    const uint32_t cstride = (uint32_t)L.cvt_stride();
 
-    int stage = 0;
+    int st = 0;
+    uint32_t ph = 0;
     bool ok = true;
     for (int rgi = 0; rgi < my_rg; ++rgi) {
-        const int p = rgi % PR;
-        ok = ok && mbar_wait(&pready[p], (rgi / PR) & 1);
-        const uint32_t cv = cbase + (uint32_t)(p * L.cvt_stride());
-        const uint32_t cva = cv + prow_a + (uint32_t)(gwarp * 8), cvb = cv + prow_b + (uint32_t)(gwarp * 8);
         float y[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int c = 0; c < nchunks; ++c, ++stage) {
-            const int st = stage % kTmaStages;
-            ok = ok && mbar_wait(&full[st], (stage / kTmaStages) & 1);
+        for (int c = 0; c < nchunks; ++c) {
+            ok = ok && mbar_wait(&full[st], ph);
             const uint32_t sb = sbase + (uint32_t)(st * kTmaStageBytes) + wrow;
+            const uint32_t cva = prow + (uint32_t)st * cstride;
             const uint32_t xb = xrow + (uint32_t)(c * kStepsPerStage * WT * 64);
-            const uint32_t gb = (uint32_t)(c * (kStepsPerStage / R) * 8);
             const uint32_t x0b = xs0 + (uint32_t)(c * kStepsPerStage * 4);
             const uint32_t x1b = xs1 + (uint32_t)(c * kStepsPerStage * 4);
             // the warp's Q k-steps as straight-line code: fragment loads, then independent
@@ -714,9 +724,9 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
 #pragma unroll
             for (int q = 0; q < Q; ++q) {
                 // fold: y += (scale16 2^24) (D1 + D16/16) - (scale16 z) sum_k x
-                const uint32_t go = gb + (uint32_t)((q / R) * 8);
+                const uint32_t go = (uint32_t)((q / R) * 8);
                 const uint2 pa = lds64(cva + go);
-                const uint2 pbv = lds64(cvb + go);
+                const uint2 pbv = lds64(cva + go + 8 * GPC * 8);
                 const float x0 = ldsf(x0b + (uint32_t)(q * 4)) * xm0;
                 const float sa = __uint_as_float(pa.x), sza = __uint_as_float(pa.y);
                 const float sb2 = __uint_as_float(pbv.x), szb = __uint_as_float(pbv.y);
@@ -730,9 +740,8 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
+            if (++st == S) { st = 0; ph ^= 1u; }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pempty[p]);
         // hand the partial sums to the reducer warp (no CTA-wide barrier)
         const int b = rgi & 1;
         if (rgi >= 2) ok = ok && mbar_wait(&rempty[b], ((rgi >> 1) - 1) & 1);
