@@ -125,15 +125,27 @@ awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const 
     return launch_status();
 }
 
-// Stages and raw parameter slots of the TMA GEMV: the deepest ring (3..6 stages) with
-// which two CTAs fit on an SM, else the deepest with which one fits; false if none fits.
-bool pick_gemv_tma(const DeviceInfo& d, int M, int K, int G, int& S, int& PR) {
-    PR = GemvTmaSmem::param_slots(K);
-    for (int ctas = 2; ctas >= 1; --ctas)
-        for (S = kTmaMaxStages; S >= kTmaMinStages; --S) {
-            const size_t b = GemvTmaSmem(M, K, G, S, PR).bytes();
-            if (b <= (size_t)d.max_smem_optin && (size_t)ctas * (b + 1024) <= (size_t)d.smem_per_sm) return true;
-        }
+// Stages and raw parameter slots of the TMA GEMV.  Parameters are small (1/32 of the
+// weight bytes at G = 128), so every row group a CTA will take gets a raw slot when
+// that fits (up to 8): all parameter copies are then issued at the start and none
+// waits behind the weight stream.  Preference: two CTAs per SM, then at least four
+// stages, then the most parameter slots, then the deepest ring (3..6 stages); false
+// if nothing fits.
+bool pick_gemv_tma(const DeviceInfo& d, int M, int N, int K, int G, int& S, int& PR, int& ctas) {
+    const int n_rg = N / kGemvRows;
+    for (ctas = 2; ctas >= 1; --ctas) {
+        const int slots = d.sms * ctas;
+        const int grid = n_rg < slots ? n_rg : slots;
+        const int per_cta = (n_rg + grid - 1) / grid;
+        const int pr_max = per_cta < kTmaMaxParamSlots ? (per_cta > 2 ? per_cta : 2) : kTmaMaxParamSlots;
+        for (int s_floor = kTmaMinStages + 1; s_floor >= kTmaMinStages; --s_floor)
+            for (PR = pr_max; PR >= 2; --PR)
+                for (S = kTmaMaxStages; S >= s_floor; --S) {
+                    const size_t b = GemvTmaSmem(M, K, G, S, PR).bytes();
+                    if (b <= (size_t)d.max_smem_optin && (size_t)ctas * (b + 1024) <= (size_t)d.smem_per_sm)
+                        return true;
+                }
+    }
     return false;
 }
 
@@ -143,8 +155,8 @@ awq_status launch_gemv_tma(const uint16_t* X, int M, const uint32_t* qweight, co
                            cudaStream_t st) {
     DeviceInfo d;
     if (!device_info(d)) return AWQ_ERR_CUDA;
-    int S = 0, PR = 0;
-    if (!pick_gemv_tma(d, M, K, G, S, PR)) return AWQ_ERR_UNSUPPORTED;
+    int S = 0, PR = 0, ctas = 0;
+    if (!pick_gemv_tma(d, M, N, K, G, S, PR, ctas)) return AWQ_ERR_UNSUPPORTED;
     const size_t smem = GemvTmaSmem(M, K, G, S, PR).bytes();
     // qweight [N][K/8] words viewed as {16 words, N rows, K/128 blocks}
     CUtensorMap tq;
@@ -187,8 +199,8 @@ awq_status dispatch_gemv(const uint16_t* X, int M, const uint32_t* qweight, cons
     if (!device_info(d)) return AWQ_ERR_CUDA;
     if (N % kGemvRows == 0 && K % 128 == 0 && (uintptr_t)scales % 16 == 0 &&
         (!cfg.zero_point || (uintptr_t)qzeros % 16 == 0)) {
-        int S = 0, PR = 0;
-        if (pick_gemv_tma(d, M, K, cfg.q_group_size, S, PR)) {
+        int S = 0, PR = 0, ctas = 0;
+        if (aligned16(X) && pick_gemv_tma(d, M, N, K, cfg.q_group_size, S, PR, ctas)) {
 #define AWQ_GEMV_TMA(GG) return launch_gemv_tma<GG, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s)
             switch (cfg.q_group_size) {
                 case 32: AWQ_GEMV_TMA(32);

@@ -366,6 +366,7 @@ constexpr int kTmaConverterWarp = kTmaConsumers + 1;        // scale/zero copies
 constexpr int kTmaReducerWarp = kTmaConsumers + 2;          // partial sums -> Y
 constexpr int kTmaThreads = (kTmaConsumers + 3) * 32;
 constexpr int kTmaMinStages = 3, kTmaMaxStages = 6;
+constexpr int kTmaMaxParamSlots = 8;
 constexpr int kTmaKC = 2048;                                // codes per row per stage
 constexpr int kTmaBlkBytes = kGemvRows * 64;               // one 128-code block of 16 rows
 constexpr int kTmaStageBytes = (kTmaKC / 128) * kTmaBlkBytes;
@@ -382,11 +383,6 @@ struct GemvTmaSmem {
         nzw = (ng + 7) / 8;
         gpc = kTmaKC / G;
     }
-    // raw parameter slots for a row group: PR = 4, 3, 2 for 1, 2-3, >= 4 stages per row
-    static __host__ __device__ int param_slots(int K) {
-        const int nchunks = (K + kTmaKC - 1) / kTmaKC;
-        return nchunks >= 4 ? 2 : (nchunks >= 2 ? 3 : 4);
-    }
     static __host__ __device__ size_t al16(size_t x) { return (x + 15) & ~(size_t)15; }
     __host__ __device__ size_t raw_scale_bytes() const { return (size_t)kGemvRows * ng * 2; }
     __host__ __device__ size_t raw_zero_bytes() const { return (size_t)kGemvRows * nzw * 4; }
@@ -399,8 +395,8 @@ struct GemvTmaSmem {
     __host__ __device__ size_t xsum() const { return x() + (size_t)M * GemvSmem::x_pitch(Kp); }
     __host__ __device__ size_t part() const { return al16(xsum() + (size_t)M * nstepsp * 4); }
     __host__ __device__ size_t bars() const { return (part() + 2 * part_stride() + 7) & ~(size_t)7; }
-    // full[S], empty[S], pfull[PR], rfull[2], rempty[2]
-    __host__ __device__ size_t bytes() const { return bars() + (2 * S + PR + 4) * 8; }
+    // full[S], empty[S], pfull[PR], rfull[2], rempty[2], xfull
+    __host__ __device__ size_t bytes() const { return bars() + (2 * S + PR + 5) * 8; }
 };
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -466,6 +462,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     uint64_t* pfull = empty + S;                // raw parameters of a row group landed
     uint64_t* rfull = pfull + PR;               // partial sums of a row group written
     uint64_t* rempty = rfull + 2;               // reducer done with a partial-sum slot
+    uint64_t* xfull = rempty + 2;               // X rows landed
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
@@ -477,6 +474,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
             mbar_init(&rfull[i], kTmaConsumers);
             mbar_init(&rempty[i], 1);
         }
+        mbar_init(xfull, 1);
         mbar_fence_init();
         prefetch_tensormap(&tmap_q);
     }
@@ -591,72 +589,51 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     }
 
     // ---------------- consumers: stage X (permuted, zero past K) and its per-step sums ----------------
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // One bulk copy per X row lands the rows unpermuted; each round then reads 256
+    // 16-byte chunks (16 whole k-steps of one row), and after a barrier writes them
+    // back in place in the order the B fragments want, while the lanes of each
+    // k-step add up its codes' activations.
     const size_t pitch = GemvSmem::x_pitch(L.Kp);
     uint8_t* xs = smem + L.x();
     float* xsum = reinterpret_cast<float*>(smem + L.xsum());
-    const int kw = L.Kp >> 3;                 // words per padded row
-    const int kwv = K >> 3;                   // words per row that hold data
     constexpr int kCons = kTmaConsumers * 32;
-    for (int u0 = threadIdx.x; u0 < M * kw; u0 += kCons * 4) {
-        uint4 v[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int u = u0 + i * kCons;
-            v[i] = make_uint4(0, 0, 0, 0);
-            if (u < M * kw) {
-                const int m = u / kw;
-                const int word = u - m * kw;
-                if (word < kwv) v[i] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)m * K + word * 8));
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int u = u0 + i * kCons;
-            if (u < M * kw) {
-                const int m = u / kw;
-                const int word = u - m * kw;
-                uint4 p;
-                p.x = __byte_perm(v[i].x, v[i].z, 0x5410);
-                p.y = __byte_perm(v[i].y, v[i].w, 0x5410);
-                p.z = __byte_perm(v[i].x, v[i].z, 0x7632);
-                p.w = __byte_perm(v[i].y, v[i].w, 0x7632);
-                const int s = word / (4 * WT);
-                const int r = word - s * 4 * WT;
-                const int tt = r / WT, j = r - tt * WT;
-                *reinterpret_cast<uint4*>(xs + m * pitch + ((size_t)(s * WT + j) * 4 + tt) * 16) = p;
-            }
-        }
+    if (threadIdx.x == 0) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        mbar_arrive_expect_tx(xfull, (uint32_t)M * (uint32_t)K * 2u);
+        for (int m = 0; m < M; ++m) bulk_g2s(xs + m * pitch, X + (size_t)m * K, (uint32_t)K * 2u, xfull);
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
+    bool ok = mbar_wait(xfull, 0);
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     {
-        // TPS threads per (row, k-step), each adding UPT 16-byte chunks, then a
-        // butterfly over the TPS lanes
-        constexpr int TPS = 4 * WT < 8 ? 4 * WT : 8;
-        constexpr int UPT = 4 * WT / TPS;
-        const int items = M * nstepsp * TPS;
-        for (int u0 = 0; u0 < items; u0 += kCons) {
+        constexpr int TPS = 4 * WT;                     // chunks (lanes) per k-step
+        const int kwp = L.Kp >> 3;                      // chunks per padded row
+        const int kwv = K >> 3;                         // chunks per row that hold data
+        for (int u0 = 0; u0 < M * kwp; u0 += kCons) {   // kwp is a multiple of kCons
             const int u = u0 + threadIdx.x;
+            const int m = u0 / kwp;
+            const int word = u - m * kwp;
+            uint4* row = reinterpret_cast<uint4*>(xs + m * pitch);
+            const uint4 v = word < kwv ? row[word] : make_uint4(0u, 0u, 0u, 0u);
+            asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
+            uint4 p;
+            p.x = __byte_perm(v.x, v.z, 0x5410);
+            p.y = __byte_perm(v.y, v.w, 0x5410);
+            p.z = __byte_perm(v.x, v.z, 0x7632);
+            p.w = __byte_perm(v.y, v.w, 0x7632);
+            const int s = word / TPS, r = word % TPS;
+            const int tt = r / WT, j = r % WT;
+            row[(s * WT + j) * 4 + tt] = p;
+            const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
             float acc = 0.0f;
-            if (u < items) {
-                const int ms = u / TPS, part = u % TPS;
-                const int m = ms / nstepsp, s = ms - m * nstepsp;
-                const uint4* xr = reinterpret_cast<const uint4*>(xs + m * pitch) + (size_t)s * WT * 4 + part * UPT;
 #pragma unroll
-                for (int i = 0; i < UPT; ++i) {
-                    const uint4 v = xr[i];
-                    const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc += h2f(h[e]);
-                }
-            }
+            for (int e = 0; e < 8; ++e) acc += h2f(h[e]);
 #pragma unroll
             for (int o = TPS / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (u < items && u % TPS == 0) xsum[u / TPS] = acc;
+            if (r == 0) xsum[m * nstepsp + s] = acc;
         }
+        // (a round writes only the chunks it read, so rounds need no barrier between them)
+        asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
 
     // ---------------- consumers: stream the stages ----------------
     // Every per-k-step shared address below is a per-stage base plus a compile-time
@@ -681,7 +658,6 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
 
     int st = 0;
     uint32_t ph = 0;
-    bool ok = true;
     for (int rgi = 0; rgi < my_rg; ++rgi) {
         float y[4] = {0.f, 0.f, 0.f, 0.f};
         for (int c = 0; c < nchunks; ++c) {
