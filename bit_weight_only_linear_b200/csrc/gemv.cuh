@@ -360,10 +360,14 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
 //     order.  Every wait is bounded.
 // ---------------------------------------------------------------------------
 
+// The helper warps take the lowest warp indices: the warp schedulers favour lower
+// indices among ready warps, and a helper that the consumers out-rank was measured to
+// fall behind (one instruction per 15-20 cycles) and stall every stage.
 constexpr int kTmaConsumers = 8;                            // consumer warps
-constexpr int kTmaProducerWarp = kTmaConsumers;             // weight TMA copies
-constexpr int kTmaConverterWarp = kTmaConsumers + 1;        // scale/zero copies -> fp32 pairs
-constexpr int kTmaReducerWarp = kTmaConsumers + 2;          // partial sums -> Y
+constexpr int kTmaProducerWarp = 0;                         // weight TMA copies
+constexpr int kTmaConverterWarp = 1;                        // scale/zero copies -> fp32 pairs
+constexpr int kTmaReducerWarp = 2;                          // partial sums -> Y
+constexpr int kTmaFirstConsumer = 3;                        // consumers: warps 3 .. 10
 constexpr int kTmaThreads = (kTmaConsumers + 3) * 32;
 constexpr int kTmaMinStages = 3, kTmaMaxStages = 6;
 constexpr int kTmaMaxParamSlots = 8;
@@ -480,9 +484,24 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     }
     __syncthreads();
 
+    // raw scales/zeros of row group j into slot j % PR (one thread)
+    const uint32_t pbytes = (uint32_t)(L.raw_scale_bytes() + (zp ? L.raw_zero_bytes() : 0));
+    auto issue_params = [&](int j) {
+        const int p = j % PR;
+        const int r0 = (blockIdx.x + j * gridDim.x) * kGemvRows;
+        uint8_t* raw = smem + L.raw() + p * L.raw_stride();
+        mbar_arrive_expect_tx(&pfull[p], pbytes);
+        bulk_g2s(raw, scales + (size_t)r0 * ng, (uint32_t)L.raw_scale_bytes(), &pfull[p]);
+        if (zp)
+            bulk_g2s(raw + L.al16(L.raw_scale_bytes()), qzeros + (size_t)r0 * nzw, (uint32_t)L.raw_zero_bytes(),
+                     &pfull[p]);
+    };
     if (warp == kTmaProducerWarp) {
-        // ---------------- producer: the weight stream, gated only by free stages ----------------
+        // ---------------- producer: the first parameter copies, then the weight stream,
+        // gated only by free stages (parameters first so that they do not queue behind
+        // the weights) ----------------
         if (lane == 0) {
+            for (int j = 0; j < PR && j < my_rg; ++j) issue_params(j);
             bool ok = true;
             int stage = 0, st = 0;
             uint32_t ph = 0;                    // parity of the current use of slot st
@@ -504,26 +523,18 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     }
     if (warp == kTmaConverterWarp) {
         // ---------------- converter: raw scales/zeros of a row group -> per-stage
-        // (scale16 * 2^24, scale16 * zero) pairs ----------------
-        const uint32_t pbytes = (uint32_t)(L.raw_scale_bytes() + (zp ? L.raw_zero_bytes() : 0));
-        auto issue_params = [&](int j) {
-            const int p = j % PR;
-            const int r0 = (blockIdx.x + j * gridDim.x) * kGemvRows;
-            uint8_t* raw = smem + L.raw() + p * L.raw_stride();
-            mbar_arrive_expect_tx(&pfull[p], pbytes);
-            bulk_g2s(raw, scales + (size_t)r0 * ng, (uint32_t)L.raw_scale_bytes(), &pfull[p]);
-            if (zp)
-                bulk_g2s(raw + L.al16(L.raw_scale_bytes()), qzeros + (size_t)r0 * nzw, (uint32_t)L.raw_zero_bytes(),
-                         &pfull[p]);
-        };
-        if (lane == 0)
-            for (int j = 0; j < PR && j < my_rg; ++j) issue_params(j);
+        // (scale16 * 2^24, scale16 * zero) pairs; refills the raw slots ----------------
         int issued = my_rg < PR ? my_rg : PR;
         bool ok = true;
         int rgi = 0, stage = 0, st = 0;
         uint32_t ph = 0;
-        constexpr int EPL = kGemvRows * GPC / 32;             // (row, group) pairs per lane per stage
-        constexpr int EB = EPL < 8 ? EPL : 8;                 // converted in batches of EB
+        // vector form: a lane takes 8 consecutive groups of one row (one 16-byte scale
+        // load, one zero word, four 16-byte stores); needs 16-byte aligned scale rows
+        const bool vec = (ng & 7) == 0;
+        constexpr int OCT = GPC / 8;                          // octets of groups per row per stage
+        constexpr int IPL = (kGemvRows * OCT + 31) / 32;      // octets per lane
+        constexpr int EPL = kGemvRows * GPC / 32;             // (row, group) pairs per lane (scalar form)
+        constexpr int EB = EPL < 8 ? EPL : 8;
         for (; rgi < my_rg && ok; ++rgi) {
             const int p = rgi % PR;
             if (!(ok = mbar_wait(&pfull[p], (rgi / PR) & 1))) break;
@@ -533,23 +544,52 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
             for (int c = 0; c < nchunks; ++c) {
                 if (stage >= S && !(ok = mbar_wait(&empty[st], ph ^ 1u))) break;
                 float2* cv = reinterpret_cast<float2*>(smem + L.cvt() + (size_t)st * L.cvt_stride());
-                for (int i0 = 0; i0 < EPL; i0 += EB) {
-                    float sc[EB];
-                    uint32_t zw[EB];
+                if (vec) {
 #pragma unroll
-                    for (int i = 0; i < EB; ++i) {
-                        const int e = lane + 32 * (i0 + i);
-                        const int r = e / GPC, grp = c * GPC + (e % GPC);
-                        const bool live = grp < ng;   // groups past K contribute nothing
-                        sc[i] = live ? h2f(rs[r * ng + grp]) : 0.0f;
-                        zw[i] = (live && zp) ? rz[r * nzw + (grp >> 3)] : 0u;
+                    for (int i = 0; i < IPL; ++i) {
+                        const int it = lane + 32 * i;
+                        if (it < kGemvRows * OCT) {
+                            const int r = it / OCT, o = it % OCT;
+                            const int g0 = c * GPC + 8 * o;
+                            uint4 v = make_uint4(0u, 0u, 0u, 0u);   // groups past K contribute nothing
+                            uint32_t zw = 0u;
+                            if (g0 < ng) {
+                                v = *reinterpret_cast<const uint4*>(rs + r * ng + g0);
+                                if (zp) zw = rz[r * nzw + (g0 >> 3)];
+                            }
+                            const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
+                            float4 out[4];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const float s0 = h2f((uint16_t)(hw[k] & 0xFFFFu)), s1 = h2f((uint16_t)(hw[k] >> 16));
+                                const float z0 = zp ? (float)((zw >> (8 * k)) & 15u) : 8.0f;
+                                const float z1 = zp ? (float)((zw >> (8 * k + 4)) & 15u) : 8.0f;
+                                out[k] = make_float4(s0 * 16777216.0f, s0 * z0, s1 * 16777216.0f, s1 * z1);
+                            }
+                            float4* dst = reinterpret_cast<float4*>(cv + r * GPC + 8 * o);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) dst[k] = out[k];
+                        }
                     }
+                } else {
+                    for (int i0 = 0; i0 < EPL; i0 += EB) {
+                        float sc[EB];
+                        uint32_t zw[EB];
 #pragma unroll
-                    for (int i = 0; i < EB; ++i) {
-                        const int e = lane + 32 * (i0 + i);
-                        const int grp = c * GPC + (e % GPC);
-                        const float z = zp ? (float)((zw[i] >> (4 * (grp & 7))) & 15u) : 8.0f;
-                        cv[e] = make_float2(sc[i] * 16777216.0f, sc[i] * z);
+                        for (int i = 0; i < EB; ++i) {
+                            const int e = lane + 32 * (i0 + i);
+                            const int r = e / GPC, grp = c * GPC + (e % GPC);
+                            const bool live = grp < ng;   // groups past K contribute nothing
+                            sc[i] = live ? h2f(rs[r * ng + grp]) : 0.0f;
+                            zw[i] = (live && zp) ? rz[r * nzw + (grp >> 3)] : 0u;
+                        }
+#pragma unroll
+                        for (int i = 0; i < EB; ++i) {
+                            const int e = lane + 32 * (i0 + i);
+                            const int grp = c * GPC + (e % GPC);
+                            const float z = zp ? (float)((zw[i] >> (4 * (grp & 7))) & 15u) : 8.0f;
+                            cv[e] = make_float2(sc[i] * 16777216.0f, sc[i] * z);
+                        }
                     }
                 }
                 __syncwarp();
@@ -589,6 +629,8 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     }
 
     // ---------------- consumers: stage X (permuted, zero past K) and its per-step sums ----------------
+    const int cw = warp - kTmaFirstConsumer;          // consumer index 0..7
+    const int ct = threadIdx.x - kTmaFirstConsumer * 32;
     // One bulk copy per X row lands the rows unpermuted; each round then reads 256
     // 16-byte chunks (16 whole k-steps of one row), and after a barrier writes them
     // back in place in the order the B fragments want, while the lanes of each
@@ -597,7 +639,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     uint8_t* xs = smem + L.x();
     float* xsum = reinterpret_cast<float*>(smem + L.xsum());
     constexpr int kCons = kTmaConsumers * 32;
-    if (threadIdx.x == 0) {
+    if (ct == 0) {
         asm volatile("griddepcontrol.wait;" ::: "memory");
         mbar_arrive_expect_tx(xfull, (uint32_t)M * (uint32_t)K * 2u);
         for (int m = 0; m < M; ++m) bulk_g2s(xs + m * pitch, X + (size_t)m * K, (uint32_t)K * 2u, xfull);
@@ -609,7 +651,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
         const int kwp = L.Kp >> 3;                      // chunks per padded row
         const int kwv = K >> 3;                         // chunks per row that hold data
         for (int u0 = 0; u0 < M * kwp; u0 += kCons) {   // kwp is a multiple of kCons
-            const int u = u0 + threadIdx.x;
+            const int u = u0 + ct;
             const int m = u0 / kwp;
             const int word = u - m * kwp;
             uint4* row = reinterpret_cast<uint4*>(xs + m * pitch);
@@ -643,17 +685,17 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     constexpr int R = G >= kStepCodes ? G / kStepCodes : 1;   // k-steps per group
     const int g = lane >> 2, t = lane & 3;
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t xrow = smem_u32(xs + (g < M ? g : 0) * pitch) + t * 16 + (uint32_t)(warp * Q * WT * 64);
+    const uint32_t xrow = smem_u32(xs + (g < M ? g : 0) * pitch) + t * 16 + (uint32_t)(cw * Q * WT * 64);
     const int m0 = 2 * t, m1 = 2 * t + 1;
-    const uint32_t xs0 = smem_u32(xsum + (m0 < M ? m0 : 0) * nstepsp) + (uint32_t)(warp * Q * 4);
-    const uint32_t xs1 = smem_u32(xsum + (m1 < M ? m1 : 0) * nstepsp) + (uint32_t)(warp * Q * 4);
+    const uint32_t xs0 = smem_u32(xsum + (m0 < M ? m0 : 0) * nstepsp) + (uint32_t)(cw * Q * 4);
+    const uint32_t xs1 = smem_u32(xsum + (m1 < M ? m1 : 0) * nstepsp) + (uint32_t)(cw * Q * 4);
     const float xm0 = m0 < M ? 1.0f : 0.0f, xm1 = m1 < M ? 1.0f : 0.0f;
     float* part = reinterpret_cast<float*>(smem + L.part());
     // weights: word w of row r in block b of a stage sits at b * kTmaBlkBytes + r * 64 + w * 4;
-    // this warp's first k-step of a stage starts a block (warp * Q is a multiple of kStepsPerBlk)
-    const uint32_t wrow = (uint32_t)((warp * Q / kStepsPerBlk) * kTmaBlkBytes + g * 64 + t * WT * 4);
+    // this warp's first k-step of a stage starts a block (cw * Q is a multiple of kStepsPerBlk)
+    const uint32_t wrow = (uint32_t)((cw * Q / kStepsPerBlk) * kTmaBlkBytes + g * 64 + t * WT * 4);
     // converted parameters of a stage: [row][group of the stage] fp32 pairs
-    const uint32_t prow = smem_u32(smem + L.cvt()) + (uint32_t)(g * GPC * 8 + ((warp * Q) / R) * 8);
+    const uint32_t prow = smem_u32(smem + L.cvt()) + (uint32_t)(g * GPC * 8 + ((cw * Q) / R) * 8);
     const uint32_t cstride = (uint32_t)L.cvt_stride();
 
     int st = 0;
@@ -721,7 +763,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
         // hand the partial sums to the reducer warp (no CTA-wide barrier)
         const int b = rgi & 1;
         if (rgi >= 2) ok = ok && mbar_wait(&rempty[b], ((rgi >> 1) - 1) & 1);
-        float* pw = part + b * (L.part_stride() / 4) + warp * kGemvRows * M;
+        float* pw = part + b * (L.part_stride() / 4) + cw * kGemvRows * M;
         if (m0 < M) {
             pw[g * M + m0] = y[0];
             pw[(g + 8) * M + m0] = y[2];

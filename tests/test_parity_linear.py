@@ -59,6 +59,23 @@ def test_gemv_outputs_do_not_spill(lib):
     assert_linear_close(b[32:32 + M * N].reshape(M, N), O.linear(X, q, sc, z, K, G, True))
 
 
+@pytest.mark.parametrize("M,K,N,G,zp", [
+    (1, 256, 47360, 128, True),     # one padded stage per row group, 10 row groups per CTA
+    (3, 2176, 38400, 32, False),    # two stages per row group (the second partial), 9 per CTA
+])
+def test_gemv_more_row_groups_than_parameter_slots(lib, M, K, N, G, zp):
+    """A CTA of the TMA GEMV keeps at most 8 row groups of raw scales/zeros in flight;
+    with more row groups per CTA than that, the slots are refilled.  Checked on every
+    output of 512 sampled rows (a spread of row groups) plus the last 16 rows."""
+    W = inputs.weights(N, K, 0.02, seed=210 + K)
+    X = inputs.activations(M, K, seed=211 + K)
+    q, sc, z, dq = _packed(W, G, zp)
+    y = _run(lib, "gemv", X, dq, G, zp)
+    rows = np.unique(np.concatenate([np.random.default_rng(212).choice(N, 512, replace=False),
+                                     np.arange(N - 16, N)]))
+    assert_linear_close(y[:, rows], O.linear_rows(X, q, sc, z, K, G, zp, rows))
+
+
 def test_gemv_single_workload_full(lib):
     """M=1, K=N=4096, G=128, zero point: every output against the oracle."""
     W = inputs.weights(4096, 4096, 0.02, seed=inputs.SEED_W)
