@@ -145,38 +145,52 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------
 
-def _dist_setup(n_gpus):
+def _dist_setup(n_gpus, backend="nccl"):
+    """Rank / world from the torchrun environment; one process group per job (NCCL on
+    the GPUs; the CPU tests use gloo).  Returns (world, rank, local_rank)."""
+    import datetime
+
     import torch
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    timeout = datetime.timedelta(seconds=120)
     if world > 1:
-        torch.cuda.set_device(local)
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local
 
 
-def _barrier(world):
+def _barrier(world, cuda=True):
     import torch
     import torch.distributed as dist
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
 
 
-def _max_over_ranks(world, value_ms):
+def _max_over_ranks(world, value_ms, device="cuda"):
+    """The slowest rank's time: every rank gets the maximum."""
     import torch
     import torch.distributed as dist
     if world == 1:
         return value_ms
-    t = torch.tensor([value_ms], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_gbs(world, bytes_per_step, steps, ms):
+    """Whole-job throughput: the bytes every rank processed over the slowest rank's
+    time (each rank runs its own copy of the work)."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
 
 
 def build_decode_layer(awq, torch, seed_offset, fused=False):
@@ -420,7 +434,7 @@ def run_ours(args):
         ms, steps = time_decode(awq, torch, layers, args.steps, args.warmup, world)
     ms = _max_over_ranks(world, ms)
     clk = clocks.summary()
-    value = world * step_bytes * steps / (ms * 1e-3) / 1e9
+    value = aggregate_gbs(world, step_bytes, steps, ms)
 
     launches = per_launch_gemv(awq, torch, layers)
     kern_bytes = sum(b for _, b, _ in launches)
@@ -432,7 +446,7 @@ def run_ours(args):
                 "peak_source": peaks["source"] + " (burst copy bandwidth)",
                 "per_linear_us": {n: round(t * 1e3, 2) for n, _, t in launches}}
     unfused_obj = {"workload": "mistral7b-layer-decode-gemv-m1-g128-zp-unfused",
-                   "value": round(world * step_bytes_7 * steps7 / (ms7 * 1e-3) / 1e9, 1), "unit": "GB/s",
+                   "value": round(aggregate_gbs(world, step_bytes_7, steps7, ms7), 1), "unit": "GB/s",
                    "ms_per_step": round(ms7 / steps7, 5), "launches_per_step": 7,
                    "per_linear_us": {n: round(t * 1e3, 2) for n, _, t in launches7}}
 
@@ -440,7 +454,7 @@ def run_ours(args):
     # note: time_decode_e2e copies each fused linear's input once per step
     e2e_ms, h2d, d2h = time_decode_e2e(awq, torch, layers, e2e_steps)
     e2e_ms = _max_over_ranks(world, e2e_ms)
-    e2e = {"value": round(world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+    e2e = {"value": round(aggregate_gbs(world, step_bytes, e2e_steps, e2e_ms), 1), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     for L in layers:
