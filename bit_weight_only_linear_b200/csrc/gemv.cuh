@@ -371,6 +371,11 @@ constexpr int kTmaFirstConsumer = 3;                        // consumers: warps 
 constexpr int kTmaThreads = (kTmaConsumers + 3) * 32;
 constexpr int kTmaMinStages = 3, kTmaMaxStages = 6;
 constexpr int kTmaMaxParamSlots = 8;
+// Weight stages a CTA requests before X has been requested.  X is the first thing the
+// consumers need and arrives only after the previous kernel has completed; a full ring
+// of weight requests issued ahead of it (up to 24 MB over the GPU) was measured to delay
+// its arrival, while two stages keep the early prefetch.
+constexpr int kTmaStagesBeforeX = 2;
 constexpr int kTmaKC = 2048;                                // codes per row per stage
 constexpr int kTmaBlkBytes = kGemvRows * 64;               // one 128-code block of 16 rows
 constexpr int kTmaStageBytes = (kTmaKC / 128) * kTmaBlkBytes;
@@ -399,8 +404,8 @@ struct GemvTmaSmem {
     __host__ __device__ size_t xsum() const { return x() + (size_t)M * GemvSmem::x_pitch(Kp); }
     __host__ __device__ size_t part() const { return al16(xsum() + (size_t)M * nstepsp * 4); }
     __host__ __device__ size_t bars() const { return (part() + 2 * part_stride() + 7) & ~(size_t)7; }
-    // full[S], empty[S], pfull[PR], rfull[2], rempty[2], xfull
-    __host__ __device__ size_t bytes() const { return bars() + (2 * S + PR + 5) * 8; }
+    // full[S], empty[S], pfull[PR], rfull[2], rempty[2], xfull, xissued
+    __host__ __device__ size_t bytes() const { return bars() + (2 * S + PR + 6) * 8; }
 };
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -467,6 +472,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     uint64_t* rfull = pfull + PR;               // partial sums of a row group written
     uint64_t* rempty = rfull + 2;               // reducer done with a partial-sum slot
     uint64_t* xfull = rempty + 2;               // X rows landed
+    uint64_t* xissued = xfull + 1;              // X copy requested
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
@@ -479,6 +485,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
             mbar_init(&rempty[i], 1);
         }
         mbar_init(xfull, 1);
+        mbar_init(xissued, 1);
         mbar_fence_init();
         prefetch_tensormap(&tmap_q);
     }
@@ -498,8 +505,9 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     };
     if (warp == kTmaProducerWarp) {
         // ---------------- producer: the first parameter copies, then the weight stream,
-        // gated only by free stages (parameters first so that they do not queue behind
-        // the weights) ----------------
+        // gated by free stages and, after kTmaStagesBeforeX stages, by the X copy having
+        // been requested (parameters and X first so that they do not queue behind the
+        // weights) ----------------
         if (lane == 0) {
             for (int j = 0; j < PR && j < my_rg; ++j) issue_params(j);
             bool ok = true;
@@ -508,6 +516,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
             for (int rgi = 0; rgi < my_rg && ok; ++rgi) {
                 const int r0 = (blockIdx.x + rgi * gridDim.x) * kGemvRows;
                 for (int c = 0; c < nchunks; ++c) {
+                    if (stage == kTmaStagesBeforeX && !(ok = mbar_wait(xissued, 0))) break;
                     if (stage >= S && !(ok = mbar_wait(&empty[st], ph ^ 1u))) break;
                     // box {16 words, 16 rows, 16 blocks}; blocks past K are filled with zeros
                     mbar_arrive_expect_tx(&full[st], kTmaStageBytes);
@@ -643,6 +652,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
         asm volatile("griddepcontrol.wait;" ::: "memory");
         mbar_arrive_expect_tx(xfull, (uint32_t)M * (uint32_t)K * 2u);
         for (int m = 0; m < M; ++m) bulk_g2s(xs + m * pitch, X + (size_t)m * K, (uint32_t)K * 2u, xfull);
+        mbar_arrive(xissued);
     }
     bool ok = mbar_wait(xfull, 0);
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
