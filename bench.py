@@ -337,17 +337,32 @@ def measure_gemm(awq, torch, reps=5):
 
 
 def measure_quantize(awq, torch, reps=20):
+    """Device time of the 4096^2 quantise/pack: a CUDA graph of `reps` calls over 10
+    rotated weight copies (10 x 32 MiB > 2x L2), timed with events on its stream (a graph,
+    so that host call overhead is not what is measured)."""
     W = torch.from_numpy(inputs.weights(4096, 4096, 0.02, inputs.SEED_W)).cuda()
-    copies = [W] + [W.clone() for _ in range(9)]        # 10 x 32 MiB rotation > 2x L2
-    outs = awq.quantize_pack(W, None, G, ZP)
+    copies = [W] + [W.clone() for _ in range(9)]
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        outs = awq.quantize_pack(W, None, G, ZP)
+        for i in range(10):
+            awq.quantize_pack(copies[i], None, G, ZP, out=outs)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(reps):
+            awq.quantize_pack(copies[i % 10], None, G, ZP, out=outs)
+    g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(reps):
-        awq.quantize_pack(copies[i % 10], None, G, ZP, out=outs)
-    e1.record()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(3):
+            g.replay()
+        e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
+    ms = e0.elapsed_time(e1) / (3 * reps)
+    del g
     nbytes = 4096 * 4096 * 2 + packed_bytes(4096, 4096)
     return {"workload": "quantize-pack-4096x4096-g128-zp", "value": round(nbytes / ms / 1e6, 1),
             "unit": "GB/s", "us": round(ms * 1e3, 2)}

@@ -287,7 +287,7 @@ awq_status awq_quantize_pack(const uint16_t* W, const uint16_t* s, int32_t N, in
     if (!W || !qweight || !scales) return AWQ_ERR_INVALID_ARG;
     if (cfg.zero_point && !qzeros) return AWQ_ERR_INVALID_ARG;
     if (!aligned16(W) || !aligned16(qweight) || (s && !aligned16(s))) return AWQ_ERR_INVALID_ARG;
-    const long long blocks = (long long)N * ceil_div(K, kQuantChunk);
+    const long long blocks = (long long)ceil_div(N, kQuantRows) * ceil_div(K, kQuantChunk);
     if (blocks > 0x7fffffffLL) return AWQ_ERR_UNSUPPORTED;
     quantize_pack_kernel<<<(unsigned)blocks, kQuantThreads, 0, (cudaStream_t)stream>>>(
         W, s, N, K, cfg.q_group_size, cfg.zero_point, qweight, scales, cfg.zero_point ? qzeros : nullptr);

@@ -18,9 +18,23 @@ constexpr float kScaleFloor = 1e-5f;
 
 struct GroupParams {
     float sc;     // fp32 value of the fp16 scale
+    float rc;     // fl(1 / sc), correctly rounded
     float zero;   // integer-valued
     uint16_t sc16;
 };
+
+// rint(fl(ws / sc)) (IEEE fp32 division, then round half to even) with the division
+// done only near a rounding boundary.  With rc = fl(1/sc) and t = fl(ws * rc), the
+// standard error model gives |t - ws/sc| <= |ws/sc| (2^-24 + 2^-24 + 2^-48), and fl(ws/sc)
+// is within |ws/sc| 2^-24 of ws/sc; so if t is farther than |t| 2^-21 from the nearest
+// half-integer, ws/sc, t and fl(ws/sc) lie strictly on the same side of it (and fl(ws/sc)
+// is no tie), and rint(t) = rint(fl(ws/sc)).  Otherwise the exact division decides.
+__device__ __forceinline__ float rint_quotient(float ws, float sc, float rc) {
+    const float t = __fmul_rn(ws, rc);
+    const float half_dist = fabsf(__fsub_rn(__fsub_rn(t, floorf(t)), 0.5f));
+    if (half_dist > fabsf(t) * 0x1p-21f) return rintf(t);
+    return rintf(__fdiv_rn(ws, sc));
+}
 
 // Per-group scale/zero from the group's extreme values, as the header defines.
 __device__ __forceinline__ GroupParams group_params(float mx, float mn, bool zero_point) {
@@ -30,13 +44,15 @@ __device__ __forceinline__ GroupParams group_params(float mx, float mn, bool zer
         scale32 = fmaxf(scale32, kScaleFloor);
         p.sc16 = f2h_rn(scale32);
         p.sc = h2f(p.sc16);
-        p.zero = fminf(fmaxf(rintf(__fdiv_rn(-mn, p.sc)), 0.0f), 15.0f);
+        p.rc = __frcp_rn(p.sc);
+        p.zero = fminf(fmaxf(rint_quotient(-mn, p.sc, p.rc), 0.0f), 15.0f);
     } else {
         float amax = fmaxf(fabsf(mx), fabsf(mn));
         float scale32 = __fdiv_rn(amax, 7.0f);
         scale32 = fmaxf(scale32, kScaleFloor);
         p.sc16 = f2h_rn(scale32);
         p.sc = h2f(p.sc16);
+        p.rc = __frcp_rn(p.sc);
         p.zero = 8.0f;
     }
     return p;
@@ -44,7 +60,7 @@ __device__ __forceinline__ GroupParams group_params(float mx, float mn, bool zer
 
 // Code of one scaled weight.
 __device__ __forceinline__ uint32_t quant_code(float ws, const GroupParams& p, bool zero_point) {
-    float r = rintf(__fdiv_rn(ws, p.sc));
+    float r = rint_quotient(ws, p.sc, p.rc);
     if (zero_point) return (uint32_t)fminf(fmaxf(r + p.zero, 0.0f), 15.0f);
     return (uint32_t)(fminf(fmaxf(r, -8.0f), 7.0f) + 8.0f);
 }
@@ -57,72 +73,86 @@ __device__ __forceinline__ void seg_minmax(float& mx, float& mn, int seg) {
     }
 }
 
-// One block per (row, 2048-channel chunk); thread t owns channels [8t, 8t+8) of the
-// chunk and writes one qweight word.  A group of G channels spans G/8 lanes of one
-// warp, so its min/max is a shuffle butterfly; the chunk holds whole zero words
-// (2048/G groups, a multiple of 8), packed through shared memory.
+// One block per (4 rows, 2048-channel chunk); thread t owns channels [8t, 8t+8) of the
+// chunk in each of the 4 rows and writes one qweight word per row.  The 4 rows' loads
+// are issued together, so their latency overlaps the quantisation of the rows before.
+// A group of G channels spans G/8 lanes of one warp, so its min/max is a shuffle
+// butterfly; the chunk holds whole zero words (2048/G groups, a multiple of 8), packed
+// through shared memory.
+constexpr int kQuantRows = 4;
+
 __global__ void __launch_bounds__(kQuantThreads)
 quantize_pack_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict__ s, int N, int K,
                      int G, int zero_point, uint32_t* __restrict__ qweight,
                      uint16_t* __restrict__ scales, uint32_t* __restrict__ qzeros) {
-    __shared__ uint8_t zbuf[kQuantChunk / 32];
+    __shared__ uint8_t zbuf[kQuantRows][kQuantChunk / 32];
     const int nchunks = ceil_div(K, kQuantChunk);
-    const int row = blockIdx.x / nchunks;
+    const int row0 = (blockIdx.x / nchunks) * kQuantRows;
     const int chunk = blockIdx.x % nchunks;
     const int k0 = chunk * kQuantChunk + threadIdx.x * 8;
     const bool active = k0 < K;
     const bool zp = zero_point != 0;
-
-    float ws[8];
-    if (active) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(W + (size_t)row * K + k0);
-        const uint16_t* wh = reinterpret_cast<const uint16_t*>(&wv);
-        if (s != nullptr) {
-            const uint4 sv = *reinterpret_cast<const uint4*>(s + k0);
-            const uint16_t* sh = reinterpret_cast<const uint16_t*>(&sv);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ws[i] = __fmul_rn(h2f(wh[i]), h2f(sh[i]));   // exact
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ws[i] = h2f(wh[i]);
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ws[i] = 0.0f;
-    }
-    float mx = ws[0], mn = ws[0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) {
-        mx = fmaxf(mx, ws[i]);
-        mn = fminf(mn, ws[i]);
-    }
-    seg_minmax(mx, mn, G >> 3);
-    const GroupParams p = group_params(mx, mn, zp);
-
     const int ng = K / G;
-    if (active) {
-        uint32_t word = 0;
+
+    uint4 wv[kQuantRows];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) word |= quant_code(ws[i], p, zp) << (4 * i);
-        qweight[(size_t)row * (K >> 3) + (k0 >> 3)] = word;
-        if ((k0 % G) == 0) {
-            const int g = k0 / G;
-            scales[(size_t)row * ng + g] = p.sc16;
-            zbuf[(threadIdx.x * 8) / G] = (uint8_t)p.zero;
+    for (int r = 0; r < kQuantRows; ++r) {
+        wv[r] = make_uint4(0u, 0u, 0u, 0u);
+        if (active && row0 + r < N) wv[r] = *reinterpret_cast<const uint4*>(W + (size_t)(row0 + r) * K + k0);
+    }
+    float sf[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sf[i] = 1.0f;
+    if (s != nullptr && active) {
+        const uint4 sv = *reinterpret_cast<const uint4*>(s + k0);
+        const uint16_t* sh = reinterpret_cast<const uint16_t*>(&sv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sf[i] = h2f(sh[i]);
+    }
+
+#pragma unroll
+    for (int r = 0; r < kQuantRows; ++r) {
+        const int row = row0 + r;                       // uniform over the block
+        const uint16_t* wh = reinterpret_cast<const uint16_t*>(&wv[r]);
+        float ws[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ws[i] = s != nullptr ? __fmul_rn(h2f(wh[i]), sf[i]) : h2f(wh[i]);   // exact
+        float mx = ws[0], mn = ws[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) {
+            mx = fmaxf(mx, ws[i]);
+            mn = fminf(mn, ws[i]);
+        }
+        seg_minmax(mx, mn, G >> 3);
+        const GroupParams p = group_params(mx, mn, zp);
+        if (active && row < N) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) word |= quant_code(ws[i], p, zp) << (4 * i);
+            qweight[(size_t)row * (K >> 3) + (k0 >> 3)] = word;
+            if ((k0 % G) == 0) {
+                const int g = k0 / G;
+                scales[(size_t)row * ng + g] = p.sc16;
+                zbuf[r][(threadIdx.x * 8) / G] = (uint8_t)p.zero;
+            }
         }
     }
     if (!zp) return;
     __syncthreads();
     const int groups_here = kQuantChunk / G;          // multiple of 8
     const int g_base = chunk * groups_here;
-    const int zw = threadIdx.x;
-    if (zw < groups_here / 8 && g_base + zw * 8 < ng) {
-        uint32_t word = 0;
-        for (int i = 0; i < 8; ++i) {
-            const int g = g_base + zw * 8 + i;
-            if (g < ng) word |= (uint32_t)zbuf[zw * 8 + i] << (4 * i);
+    const int words = groups_here / 8;
+    for (int t = threadIdx.x; t < kQuantRows * words; t += kQuantThreads) {
+        const int r = t / words, zw = t - r * words;
+        const int row = row0 + r;
+        if (row < N && g_base + zw * 8 < ng) {
+            uint32_t word = 0;
+            for (int i = 0; i < 8; ++i) {
+                const int g = g_base + zw * 8 + i;
+                if (g < ng) word |= (uint32_t)zbuf[r][zw * 8 + i] << (4 * i);
+            }
+            qzeros[(size_t)row * ceil_div(ng, 8) + (g_base >> 3) + zw] = word;
         }
-        qzeros[(size_t)row * ceil_div(ng, 8) + (g_base >> 3) + zw] = word;
     }
 }
 

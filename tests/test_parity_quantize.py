@@ -48,6 +48,27 @@ def test_quantize_pack_edge_values(lib):
             _check(lib, W, None, G, zp)
 
 
+def test_quantize_pack_round_half_even_ties(lib):
+    """Quotients w/scale that land exactly on half-integers (the scale is 2^-7, every
+    weight an odd multiple of 2^-8): the codes must follow round-half-to-even of the IEEE
+    quotient, which the kernel decides with an exact division near rounding boundaries."""
+    K = 256
+    u = 2.0 ** -7
+    ties_zp = np.array([0.0, 15 * u] + [(k % 15 + 0.5) * u for k in range(K - 2)])
+    ties_sym = np.array([-7 * u, 7 * u] + [((k % 15) - 7.5) * u for k in range(K - 2)])
+    ties_sym = np.clip(ties_sym, -7 * u, 7 * u)
+    for G in O.GROUP_SIZES:
+        # every group holds the extremes that fix the scale at 2^-7, then the ties
+        def grouped(base):
+            out = np.empty(K)
+            for g0 in range(0, K, G):
+                out[g0:g0 + G] = np.concatenate([base[:2], base[2:2 + G - 2]])
+            return out
+        W = np.stack([grouped(ties_zp), grouped(ties_zp)[::-1].copy(), grouped(ties_sym)]).astype(np.float16)
+        for zp in (True, False):
+            _check(lib, W, None, G, zp)
+
+
 def test_quantize_pack_full_layer_4096(lib):
     """The 4096 x 4096 layer of the single-GEMV workload, every element."""
     W = inputs.weights(4096, 4096, 0.02, seed=inputs.SEED_W)
