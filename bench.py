@@ -72,8 +72,7 @@ def profile_traffic(kernel_tag: str):
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
-    from bit_weight_only_linear_b200 import build
-    digest = source_digest(build.sources())
+    digest = source_digest(gemv_sources())
     for line in open(path):
         parts = line.split()
         if len(parts) >= 3 and parts[0] == kernel_tag and not line.startswith("#"):
@@ -81,6 +80,14 @@ def profile_traffic(kernel_tag: str):
                 return None
             return float(parts[1])
     return None
+
+
+def gemv_sources():
+    """The files that define the decode GEMV kernel and its launch configuration: a
+    recorded traffic figure stays valid while none of them changes."""
+    from bit_weight_only_linear_b200 import build
+    names = ("gemv.cuh", "sm100.cuh", "common.cuh", "awq_api.cu")
+    return [p for p in build.sources() if os.path.basename(p) in names]
 
 
 def source_digest(paths) -> str:

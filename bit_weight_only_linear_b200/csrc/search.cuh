@@ -7,7 +7,8 @@
 // awq_quantize_pack, the rest in fp64):
 //   m_k    = mean_t |X[t][k]|                       (exact: fp64 sums of fp16 values)
 //   s_k    = fp16(max(pow(m_k, alpha), 2^-14))
-//   dW     = (Q(W s) - W s) / s  = Q(W s)/s - W      (per element, fp64, kept as fp32)
+//   dW     = (Q(W s) - W s) / s  = Q(W s)/s - W      (difference exact in fp64, quotient
+//                                                      in fp32: within one fp32 ulp)
 //   loss   = mean_{t,n} (sum_k X[t][k] dW[n][k])^2
 // The loss GEMM E = X dW^T is a dense contraction and runs on tcgen05: dW of each
 // row n is scaled by 2^e_n (its largest entry lands in [2^13, 2^14)) and split into
@@ -115,8 +116,9 @@ search_delta_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict__
             for (int i = 0; i < 8; ++i) {
                 const float q = (float)quant_code(ws[i], p, zp);
                 const float deq = __fmul_rn(q - p.zero, p.sc);                        // exact
-                const double d = __ddiv_rn((double)deq - (double)ws[i], (double)sv[i]);  // exact difference
-                const float df = (float)d;
+                // fp32 quotient of the fp64-exact difference: within one fp32 ulp of the
+                // correctly rounded dW, far below the 22-bit hi/lo split that follows
+                const float df = __fdiv_rn((float)((double)deq - (double)ws[i]), sv[i]);
                 dsm[k0 + i] = df;
                 amax = fmaxf(amax, fabsf(df));
             }
@@ -145,13 +147,24 @@ search_delta_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict__
     // last block (k >= K) is written as zeros
     const int kp = search_kp(K);
     uint16_t* out = dw + ((size_t)a * N + row) * (size_t)(2 * kp);
-    for (int k = threadIdx.x; k < kp; k += kQuantThreads) {
-        const float v = k < K ? ldexpf(dsm[k], e) : 0.0f;
-        const uint16_t hi = f2h_rn(v);
-        const uint16_t lo = f2h_rn(v - h2f(hi));     // exact difference
-        const int kb = k >> 6, w = k & 63;
-        out[kb * 128 + w] = hi;
-        out[kb * 128 + 64 + w] = lo;
+    for (int k0 = threadIdx.x * 8; k0 < kp; k0 += kQuantThreads * 8) {   // 8 channels, 16-byte stores
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            uint16_t h2[2], l2[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int k = k0 + i + j;
+                const float v = k < K ? ldexpf(dsm[k], e) : 0.0f;
+                h2[j] = f2h_rn(v);
+                l2[j] = f2h_rn(v - h2f(h2[j]));   // exact difference
+            }
+            hw[i / 2] = (uint32_t)h2[0] | ((uint32_t)h2[1] << 16);
+            lw[i / 2] = (uint32_t)l2[0] | ((uint32_t)l2[1] << 16);
+        }
+        const int kb = k0 >> 6, w = k0 & 63;
+        *reinterpret_cast<uint4*>(out + kb * 128 + w) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(out + kb * 128 + 64 + w) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
 }
 
