@@ -91,10 +91,16 @@ def gemv_sources():
 
 
 def source_digest(paths) -> str:
+    """Digest of the code in `paths`: comments and blank lines do not count, so that a
+    comment edit does not invalidate a recorded measurement."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for p in sorted(paths):
-        h.update(open(p, "rb").read())
+        text = open(p, encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln).encode())
     return h.hexdigest()[:16]
 
 

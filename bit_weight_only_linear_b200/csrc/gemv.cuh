@@ -346,10 +346,11 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
 //     [block][row][64 B], so the two rows a quarter-warp reads are adjacent and the
 //     shared loads are conflict-free (row-major stages gave 8-way conflicts).
 //     Measured on B200: 16 per-row bulk copies per stage cap the copy rate near
-//     2 TB/s; one tensor copy per stage does not.  The producer waits for nothing
-//     but a free stage.
+//     2 TB/s; one tensor copy per stage does not.  The producer waits for a free
+//     stage and, once, for the X copy to have been requested (see kTmaStagesBeforeX).
 //   * Scales and zero words of a row group arrive through two bulk copies into a
-//     ring of PR raw parameter slots.  A converter warp turns the groups of each
+//     ring of PR raw parameter slots, all issued by the producer before its first
+//     weight stage when they fit.  A converter warp turns the groups of each
 //     stage into fp32 pairs (scale16 * 2^24, scale16 * zero) in a small buffer that
 //     belongs to the stage: a stage is full when both its TMA bytes and the
 //     converter's arrival are in, and both refill it after the consumers release
@@ -360,9 +361,7 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
 //     order.  Every wait is bounded.
 // ---------------------------------------------------------------------------
 
-// The helper warps take the lowest warp indices: the warp schedulers favour lower
-// indices among ready warps, and a helper that the consumers out-rank was measured to
-// fall behind (one instruction per 15-20 cycles) and stall every stage.
+// Warp roles: producer, converter and reducer are warps 0-2, the consumers warps 3-10.
 constexpr int kTmaConsumers = 8;                            // consumer warps
 constexpr int kTmaProducerWarp = 0;                         // weight TMA copies
 constexpr int kTmaConverterWarp = 1;                        // scale/zero copies -> fp32 pairs
