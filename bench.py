@@ -86,7 +86,7 @@ def gemv_sources():
     """The files that define the decode GEMV kernel and its launch configuration: a
     recorded traffic figure stays valid while none of them changes."""
     from bit_weight_only_linear_b200 import build
-    names = ("gemv.cuh", "sm100.cuh", "common.cuh", "awq_api.cu")
+    names = ("gemv.cuh", "sm100.cuh", "common.cuh", "launch.cuh", "awq_api.cu")
     return [p for p in build.sources() if os.path.basename(p) in names]
 
 
@@ -290,21 +290,30 @@ def per_launch_gemv(awq, torch, layers, reps=64):
 
 
 def time_decode_e2e(awq, torch, layers, steps):
-    """Same metric through the C ABI with host buffers: every step copies the 7 input
-    vectors host->device (pinned) and the 7 outputs device->host."""
-    xs_host = [torch.from_numpy(L["x_host"]).pin_memory() for L in layers]
-    ys_host = [torch.empty((1, L["N"]), dtype=torch.float16).pin_memory() for L in layers]
-    h2d = sum(x.numel() * 2 for x in xs_host)
-    d2h = sum(y.numel() * 2 for y in ys_host)
+    """Same metric through the C ABI with host buffers: every step copies the layer's
+    input vectors host->device (one copy from one pinned buffer), runs the GEMV calls,
+    and copies their outputs device->host (one copy into one pinned buffer)."""
+    ks = [L["K"] for L in layers]
+    ns = [L["N"] for L in layers]
+    x_host = torch.from_numpy(np.concatenate([L["x_host"].reshape(-1) for L in layers])).pin_memory()
+    y_host = torch.empty(sum(ns), dtype=torch.float16).pin_memory()
+    x_dev = torch.empty_like(x_host, device="cuda")
+    y_dev = torch.empty(sum(ns), dtype=torch.float16, device="cuda")
+    xo = np.cumsum([0] + ks)
+    yo = np.cumsum([0] + ns)
+    xs = [x_dev[xo[i]:xo[i + 1]].view(1, ks[i]) for i in range(len(layers))]   # 16-byte aligned views
+    ys = [y_dev[yo[i]:yo[i + 1]].view(1, ns[i]) for i in range(len(layers))]
+    h2d = x_host.numel() * 2
+    d2h = y_host.numel() * 2
     s = torch.cuda.current_stream()
 
     def step(i):
         r = i % ROTATIONS
-        for L, xh, yh in zip(layers, xs_host, ys_host):
-            L["x"].copy_(xh, non_blocking=True)
+        x_dev.copy_(x_host, non_blocking=True)
+        for L, x, y in zip(layers, xs, ys):
             q, sc, z = L["copies"][r]
-            awq.linear_gemv(L["x"], q, sc, z, G, ZP, out=L["y"])
-            yh.copy_(L["y"], non_blocking=True)
+            awq.linear_gemv(x, q, sc, z, G, ZP, out=y)
+        y_host.copy_(y_dev, non_blocking=True)
 
     for i in range(8):
         step(i)

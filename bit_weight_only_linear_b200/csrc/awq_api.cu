@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "launch.cuh"
 #include "gemv.cuh"
 #include "quantize.cuh"
 #include "gemm_sm100.cuh"
@@ -94,12 +95,8 @@ awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const 
     const size_t smem = GemvSmem::bytes(M, K, nsteps);
     if (smem > (size_t)d.max_smem_optin) return AWQ_ERR_UNSUPPORTED;
     auto kern = gemv_mma_kernel<WT, ONE>;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return AWQ_ERR_CUDA;
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvThreads, smem) != cudaSuccess || occ < 1)
-        return AWQ_ERR_CUDA;
+    if (!kernel_occupancy((const void*)kern, kGemvThreads, smem, occ) || occ < 1) return AWQ_ERR_CUDA;
     // persistent grid: at most one wave, row-group iterations spread evenly over the CTAs
     constexpr int UK = kGemvUnitWords / WT;
     const int units = ceil_div(nsteps, UK);
@@ -164,11 +161,8 @@ awq_status launch_gemv_tma(const uint16_t* X, int M, const uint32_t* qweight, co
                       (uint64_t)K / 2, 64, 16, kGemvRows, kTmaKC / 128))
         return AWQ_ERR_CUDA;
     auto kern = gemv_tma_kernel<G, ONE>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return AWQ_ERR_CUDA;
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kTmaThreads, smem) != cudaSuccess || occ < 1)
-        return AWQ_ERR_CUDA;
+    if (!kernel_occupancy((const void*)kern, kTmaThreads, smem, occ) || occ < 1) return AWQ_ERR_CUDA;
     // one CTA per resident slot, row groups dealt round-robin
     const int n_rg = N / kGemvRows;
     const int slots = d.sms * occ;
