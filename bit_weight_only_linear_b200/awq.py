@@ -52,6 +52,7 @@ SIGNATURES = {
     "awq_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                               QuantConfig]),
     "awq_device_error": (ctypes.c_int, [ctypes.c_void_p]),
+    "awq_check_bounded_wait": (ctypes.c_int, [ctypes.c_void_p]),
 }
 
 _lib = None
@@ -216,6 +217,12 @@ def scale_search_noalloc(X: torch.Tensor, W: torch.Tensor, group_size: int = 128
         _dev(s_out, "s_out", _F16), losses.data_ptr(), best.data_ptr(), _stream(stream))
     _check("awq_scale_search_noalloc", st)
     return s_out, losses, best
+
+
+def check_bounded_wait(stream=None) -> None:
+    """awq_check_bounded_wait: enqueue a kernel whose wait can never complete (it gives up
+    after the library's 2 s limit and flags a timeout, read by device_error())."""
+    _check("awq_check_bounded_wait", load_library().awq_check_bounded_wait(_stream(stream)))
 
 
 def device_error(stream=None) -> None:

@@ -369,6 +369,11 @@ awq_status awq_scale_search_noalloc(const uint16_t* X, int32_t M, const uint16_t
                                     best_index_out, L, (cudaStream_t)stream);
 }
 
+awq_status awq_check_bounded_wait(void* stream) {
+    awq::sm100::bounded_wait_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
+    return launch_status();
+}
+
 awq_status awq_device_error(void* stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return AWQ_ERR_CUDA;
     unsigned word = 0, zero = 0;

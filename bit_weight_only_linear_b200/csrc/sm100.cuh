@@ -65,6 +65,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// A wait that cannot complete: one thread waits on a fresh mbarrier that nothing
+// arrives on, so the bounded wait gives up after kWaitLimitNs and raises the timeout
+// flag (awq_check_bounded_wait).
+__global__ void bounded_wait_probe_kernel() {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+        (void)mbar_wait(&bar, 0);
+    }
+}
+
 // ----------------------------------------------------------------------------
 // TMA (tile mode, no multicast)
 // ----------------------------------------------------------------------------

@@ -183,6 +183,17 @@ size_t awq_workspace_bytes(int32_t op, int32_t M, int32_t N, int32_t K, awq_quan
  */
 awq_status awq_device_error(void* stream);
 
+/*
+ * Diagnostic of the bounded device waits: enqueues on `stream` one small kernel whose
+ * mbarrier wait can never complete (nothing arrives on the barrier).  The wait gives
+ * up after the library's limit (2 s), the kernel sets the device error word and
+ * returns, so the next awq_device_error() reports AWQ_ERR_TIMEOUT and the context
+ * stays usable.  Lets a caller check, on its GPU, that a stalled pipeline of this
+ * library ends with an error status instead of a hang.  No counterpart in the pages.
+ * Returns AWQ_OK once enqueued, AWQ_ERR_CUDA if the launch fails.
+ */
+awq_status awq_check_bounded_wait(void* stream);
+
 #ifdef __cplusplus
 }
 #endif
