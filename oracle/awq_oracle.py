@@ -14,7 +14,7 @@ What it follows
   asymmetric with an offset, off = symmetric quantization).
 * "Optimization Awq" (skillsdirectory.com), quantization-config block:
   ``{"zero_point", "q_group_size", "w_bit": 4, "version"}``.
-* The task specification fixes what the pages leave open: scale = (max-min)/15,
+* The quantiser's remaining arithmetic, which the pages leave open: scale = (max-min)/15,
   zero = clamp(round(-min/scale), 0, 15), q = clamp(round_half_even(w/scale) +
   zero, 0, 15) in fp32, dequant (q - zero)*scale, fp64 matmul, s = mean|X|^alpha
   over an alpha grid, int4 codes packed 8 per uint32.

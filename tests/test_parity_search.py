@@ -1,6 +1,6 @@
 """GPU parity: awq_scale_search against the oracle's grid search.
 
-Rules (from the benchmark spec of the method and the arithmetic of the kernels):
+Rules (from the method's definition and the arithmetic of the kernels):
   * the chosen alpha index equals the oracle's, or differs by one grid step where the
     oracle's two losses differ by less than 1e-6 relative;
   * s* is bit-exact when the indices agree (both sides round pow(m, alpha) once to fp16;
