@@ -18,7 +18,9 @@ from .build import LIB
 AWQ_OK = 0
 AWQ_OP_QUANTIZE_PACK, AWQ_OP_SCALE_SEARCH, AWQ_OP_GEMV, AWQ_OP_GEMM = 0, 1, 2, 3
 STATUS_NAMES = {0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_UNSUPPORTED", 3: "AWQ_ERR_WORKSPACE",
-                4: "AWQ_ERR_CUDA", 5: "AWQ_ERR_TIMEOUT"}
+                4: "AWQ_ERR_CUDA", 5: "AWQ_ERR_TIMEOUT", 6: "AWQ_ERR_RANGE"}
+(AWQ_ERR_INVALID_ARG, AWQ_ERR_UNSUPPORTED, AWQ_ERR_WORKSPACE, AWQ_ERR_CUDA, AWQ_ERR_TIMEOUT,
+ AWQ_ERR_RANGE) = 1, 2, 3, 4, 5, 6
 
 # Every symbol the header declares, with its ctypes signature.
 _u16p = ctypes.c_void_p

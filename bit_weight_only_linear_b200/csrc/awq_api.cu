@@ -6,6 +6,7 @@
 
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "launch.cuh"
@@ -85,43 +86,6 @@ awq_status check_linear(const uint16_t* X, int M, const uint32_t* qweight, const
     return AWQ_OK;
 }
 
-template <int WT, bool ONE>
-awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
-                       const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
-                       cudaStream_t st) {
-    DeviceInfo d;
-    if (!device_info(d)) return AWQ_ERR_CUDA;
-    const int nsteps = K / (32 * WT);
-    const size_t smem = GemvSmem::bytes(M, K, nsteps);
-    if (smem > (size_t)d.max_smem_optin) return AWQ_ERR_UNSUPPORTED;
-    auto kern = gemv_mma_kernel<WT, ONE>;
-    int occ = 0;
-    if (!kernel_occupancy((const void*)kern, kGemvThreads, smem, occ) || occ < 1) return AWQ_ERR_CUDA;
-    // persistent grid: at most one wave, row-group iterations spread evenly over the CTAs
-    constexpr int UK = kGemvUnitWords / WT;
-    const int units = ceil_div(nsteps, UK);
-    const int slots = d.sms * occ;
-    const int ks = gemv_ks(units, ceil_div(N, kGemvRows), slots);
-    const int rpi = kGemvWarps / ks;
-    const int n_it = ceil_div(ceil_div(N, kGemvRows), rpi);
-    const int per_cta = ceil_div(n_it, slots);
-    const int grid = ceil_div(n_it, per_cta);
-    cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3(grid);
-    lc.blockDim = dim3(kGemvThreads);
-    lc.dynamicSmemBytes = smem;
-    lc.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    lc.attrs = attr;
-    lc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&lc, kern, X, M, qweight, scales, qzeros, N, K, (int)cfg.q_group_size,
-                           (int)cfg.zero_point, ks, Y) != cudaSuccess)
-        return AWQ_ERR_CUDA;
-    return launch_status();
-}
-
 // Stages and raw parameter slots of the TMA GEMV.  Parameters are small (1/32 of the
 // weight bytes at G = 128), so every row group a CTA will take gets a raw slot when
 // that fits (up to 8): all parameter copies are then issued at the start and none
@@ -146,70 +110,160 @@ bool pick_gemv_tma(const DeviceInfo& d, int M, int N, int K, int G, int& S, int&
     return false;
 }
 
-template <int G, bool ONE>
-awq_status launch_gemv_tma(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
-                           const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
-                           cudaStream_t st) {
+// ---------------------------------------------------------------------------
+// GEMV launch plans.  Everything a launch needs that depends only on the device and
+// on (M, N, K, G) -- which kernel, its stages and parameter slots, grid and shared
+// memory -- is worked out on the first call and cached, and so is the TMA view of
+// each weight matrix (per device, qweight pointer, N and K).  A later call makes one
+// lookup under one lock, then the launch.
+// ---------------------------------------------------------------------------
+struct GemvPlan {
+    int dev, M, N, K, G;
+    bool tma;          // TMA-staged kernel, else the register-ring kernel
+    const void* fn;
+    int grid, S, PR, ks;
+    size_t smem;
+};
+
+struct GemvTmap {
+    int dev;
+    const void* base;
+    int N, K;
+    CUtensorMap map;
+};
+
+constexpr int kGemvTmapCache = 256;
+std::vector<GemvPlan> g_gemv_plans;
+GemvTmap g_gemv_tmaps[kGemvTmapCache];
+int g_gemv_tmap_count = 0, g_gemv_tmap_next = 0;
+
+const void* gemv_tma_fn(int G, bool one) {
+    switch (G) {
+        case 32: return one ? (const void*)gemv_tma_kernel<32, true> : (const void*)gemv_tma_kernel<32, false>;
+        case 64: return one ? (const void*)gemv_tma_kernel<64, true> : (const void*)gemv_tma_kernel<64, false>;
+        case 128: return one ? (const void*)gemv_tma_kernel<128, true> : (const void*)gemv_tma_kernel<128, false>;
+        default: return one ? (const void*)gemv_tma_kernel<256, true> : (const void*)gemv_tma_kernel<256, false>;
+    }
+}
+
+const void* gemv_mma_fn(int WT, bool one) {
+    switch (WT) {
+        case 1: return one ? (const void*)gemv_mma_kernel<1, true> : (const void*)gemv_mma_kernel<1, false>;
+        case 2: return one ? (const void*)gemv_mma_kernel<2, true> : (const void*)gemv_mma_kernel<2, false>;
+        default: return one ? (const void*)gemv_mma_kernel<4, true> : (const void*)gemv_mma_kernel<4, false>;
+    }
+}
+
+// Fills p (keyed fields set by the caller).  The TMA kernel takes every shape with whole
+// 16-row groups and whole 128-code blocks whose staging fits; the register-ring kernel
+// takes the rest.
+awq_status build_gemv_plan(GemvPlan& p) {
     DeviceInfo d;
     if (!device_info(d)) return AWQ_ERR_CUDA;
     int S = 0, PR = 0, ctas = 0;
-    if (!pick_gemv_tma(d, M, N, K, G, S, PR, ctas)) return AWQ_ERR_UNSUPPORTED;
-    const size_t smem = GemvTmaSmem(M, K, G, S, PR).bytes();
+    if (p.N % kGemvRows == 0 && p.K % 128 == 0 && pick_gemv_tma(d, p.M, p.N, p.K, p.G, S, PR, ctas)) {
+        p.tma = true;
+        p.fn = gemv_tma_fn(p.G, p.M == 1);
+        p.S = S;
+        p.PR = PR;
+        p.ks = 0;
+        p.smem = GemvTmaSmem(p.M, p.K, p.G, S, PR).bytes();
+        int occ = 0;
+        if (!kernel_occupancy(p.fn, kTmaThreads, p.smem, occ) || occ < 1) return AWQ_ERR_CUDA;
+        // one CTA per resident slot, row groups dealt round-robin
+        const int n_rg = p.N / kGemvRows;
+        const int slots = d.sms * occ;
+        p.grid = n_rg < slots ? n_rg : slots;
+        return AWQ_OK;
+    }
+    p.tma = false;
+    const int WT = gemv_words_per_thread(p.G);
+    p.fn = gemv_mma_fn(WT, p.M == 1);
+    const int nsteps = p.K / (32 * WT);
+    p.smem = GemvSmem::bytes(p.M, p.K, nsteps);
+    if (p.smem > (size_t)d.max_smem_optin) return AWQ_ERR_UNSUPPORTED;
+    int occ = 0;
+    if (!kernel_occupancy(p.fn, kGemvThreads, p.smem, occ) || occ < 1) return AWQ_ERR_CUDA;
+    // persistent grid: at most one wave, row-group iterations spread evenly over the CTAs
+    const int UK = kGemvUnitWords / WT;
+    const int units = ceil_div(nsteps, UK);
+    const int slots = d.sms * occ;
+    p.ks = gemv_ks(units, ceil_div(p.N, kGemvRows), slots);
+    const int rpi = kGemvWarps / p.ks;
+    const int n_it = ceil_div(ceil_div(p.N, kGemvRows), rpi);
+    const int per_cta = ceil_div(n_it, slots);
+    p.grid = ceil_div(n_it, per_cta);
+    p.S = p.PR = 0;
+    return AWQ_OK;
+}
+
+// The cached plan for (current device, M, N, K, G) and, for the TMA kernel, the cached
+// view of qweight.
+awq_status gemv_plan(const uint32_t* qweight, int M, int N, int K, int G, GemvPlan& out, CUtensorMap& tq) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    const GemvPlan* found = nullptr;
+    for (const GemvPlan& p : g_gemv_plans)
+        if (p.dev == dev && p.M == M && p.N == N && p.K == K && p.G == G) {
+            found = &p;
+            break;
+        }
+    if (!found) {
+        GemvPlan p = {};
+        p.dev = dev, p.M = M, p.N = N, p.K = K, p.G = G;
+        const awq_status st = build_gemv_plan(p);
+        if (st != AWQ_OK) return st;
+        g_gemv_plans.push_back(p);
+        found = &g_gemv_plans.back();
+    }
+    out = *found;
+    if (!out.tma) return AWQ_OK;
+    for (int i = 0; i < g_gemv_tmap_count; ++i) {
+        const GemvTmap& e = g_gemv_tmaps[i];
+        if (e.dev == dev && e.base == qweight && e.N == N && e.K == K) {
+            tq = e.map;
+            return AWQ_OK;
+        }
+    }
     // qweight [N][K/8] words viewed as {16 words, N rows, K/128 blocks}
-    CUtensorMap tq;
     if (!make_tmap_3d(&tq, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 16, (uint64_t)N, (uint64_t)(K / 128),
                       (uint64_t)K / 2, 64, 16, kGemvRows, kTmaKC / 128))
         return AWQ_ERR_CUDA;
-    auto kern = gemv_tma_kernel<G, ONE>;
-    int occ = 0;
-    if (!kernel_occupancy((const void*)kern, kTmaThreads, smem, occ) || occ < 1) return AWQ_ERR_CUDA;
-    // one CTA per resident slot, row groups dealt round-robin
-    const int n_rg = N / kGemvRows;
-    const int slots = d.sms * occ;
-    const int grid = n_rg < slots ? n_rg : slots;
+    const int slot = g_gemv_tmap_count < kGemvTmapCache ? g_gemv_tmap_count++ : (g_gemv_tmap_next++ % kGemvTmapCache);
+    g_gemv_tmaps[slot] = {dev, qweight, N, K, tq};
+    return AWQ_OK;
+}
+
+awq_status launch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
+                       const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
+                       cudaStream_t st) {
+    GemvPlan p;
+    CUtensorMap tq;
+    const awq_status ps = gemv_plan(qweight, M, N, K, cfg.q_group_size, p, tq);
+    if (ps != AWQ_OK) return ps;
     cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3(grid);
-    lc.blockDim = dim3(kTmaThreads);
-    lc.dynamicSmemBytes = smem;
+    lc.gridDim = dim3(p.grid);
+    lc.blockDim = dim3(p.tma ? kTmaThreads : kGemvThreads);
+    lc.dynamicSmemBytes = p.smem;
     lc.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&lc, kern, tq, X, M, scales, qzeros, N, K, (int)cfg.zero_point, Y, S, PR) !=
-        cudaSuccess)
-        return AWQ_ERR_CUDA;
-    return launch_status();
-}
-
-template <bool ONE>
-awq_status dispatch_gemv(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
-                         const uint32_t* qzeros, int N, int K, const awq_quant_config& cfg, uint16_t* Y,
-                         cudaStream_t s) {
-    // every row group full, K in whole 128-code blocks, parameters 16-byte aligned and
-    // the staging fits: TMA path
-    DeviceInfo d;
-    if (!device_info(d)) return AWQ_ERR_CUDA;
-    if (N % kGemvRows == 0 && K % 128 == 0 && (uintptr_t)scales % 16 == 0 &&
-        (!cfg.zero_point || (uintptr_t)qzeros % 16 == 0)) {
-        int S = 0, PR = 0, ctas = 0;
-        if (aligned16(X) && pick_gemv_tma(d, M, N, K, cfg.q_group_size, S, PR, ctas)) {
-#define AWQ_GEMV_TMA(GG) return launch_gemv_tma<GG, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s)
-            switch (cfg.q_group_size) {
-                case 32: AWQ_GEMV_TMA(32);
-                case 64: AWQ_GEMV_TMA(64);
-                case 128: AWQ_GEMV_TMA(128);
-                default: AWQ_GEMV_TMA(256);
-            }
-#undef AWQ_GEMV_TMA
-        }
+    int zp = cfg.zero_point, G = cfg.q_group_size;
+    cudaError_t e;
+    if (p.tma) {
+        // (tmap_q, X, M, scales, qzeros, N, K, zero_point, Y, S, PR)
+        void* args[] = {&tq, &X, &M, &scales, &qzeros, &N, &K, &zp, &Y, &p.S, &p.PR};
+        e = cudaLaunchKernelExC(&lc, p.fn, args);
+    } else {
+        // (X, M, qweight, scales, qzeros, N, K, G, zero_point, ks, Y)
+        void* args[] = {&X, &M, &qweight, &scales, &qzeros, &N, &K, &G, &zp, &p.ks, &Y};
+        e = cudaLaunchKernelExC(&lc, p.fn, args);
     }
-    switch (cfg.q_group_size) {
-        case 32: return launch_gemv<1, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-        case 64: return launch_gemv<2, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-        default: return launch_gemv<4, ONE>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
-    }
+    return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
@@ -266,11 +320,12 @@ const char* awq_status_string(awq_status s) {
         case AWQ_ERR_WORKSPACE: return "AWQ_ERR_WORKSPACE: workspace too small";
         case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA: a CUDA call or kernel launch failed";
         case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT: a bounded device wait ran out";
+        case AWQ_ERR_RANGE: return "AWQ_ERR_RANGE: a dequantised weight of the fp16 GEMM path is not finite in fp16";
     }
     return "AWQ_ERR_UNKNOWN";
 }
 
-int32_t awq_abi_version(void) { return 1; }
+int32_t awq_abi_version(void) { return 2; }
 
 awq_status awq_quantize_pack(const uint16_t* W, const uint16_t* s, int32_t N, int32_t K, awq_quant_config cfg,
                              uint32_t* qweight, uint16_t* scales, uint32_t* qzeros, void* stream) {
@@ -285,6 +340,7 @@ awq_status awq_quantize_pack(const uint16_t* W, const uint16_t* s, int32_t N, in
     if (blocks > 0x7fffffffLL) return AWQ_ERR_UNSUPPORTED;
     quantize_pack_kernel<<<(unsigned)blocks, kQuantThreads, 0, (cudaStream_t)stream>>>(
         W, s, N, K, cfg.q_group_size, cfg.zero_point, qweight, scales, cfg.zero_point ? qzeros : nullptr);
+    stream_order_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
     return launch_status();
 }
 
@@ -309,9 +365,7 @@ awq_status awq_linear_gemv(const uint16_t* X, int32_t M, const uint32_t* qweight
     awq_status st = check_linear(X, M, qweight, scales, qzeros, N, K, cfg, Y);
     if (st != AWQ_OK) return st;
     if (M > 8) return AWQ_ERR_UNSUPPORTED;
-    cudaStream_t s = (cudaStream_t)stream;
-    return M == 1 ? dispatch_gemv<true>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s)
-                  : dispatch_gemv<false>(X, M, qweight, scales, qzeros, N, K, cfg, Y, s);
+    return launch_gemv(X, M, qweight, scales, qzeros, N, K, cfg, Y, (cudaStream_t)stream);
 }
 
 awq_status awq_linear_gemm(const uint16_t* X, int32_t M, const uint32_t* qweight, const uint16_t* scales,
@@ -380,7 +434,7 @@ awq_status awq_device_error(void* stream) {
     if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return AWQ_ERR_CUDA;
     if (word == 0) return AWQ_OK;
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return AWQ_ERR_CUDA;
-    return AWQ_ERR_TIMEOUT;
+    return (word & kErrTimeout) ? AWQ_ERR_TIMEOUT : AWQ_ERR_RANGE;
 }
 
 }  // extern "C"

@@ -10,8 +10,10 @@
 
 namespace awq {
 
-// Bit set in the device error word when a bounded wait runs out.
+// Bits of the device error word: a bounded wait ran out; a dequantised weight of the
+// fp16 GEMM path would not be finite in fp16 ((q - zero) * scale16 >= 65520 in magnitude).
 constexpr unsigned kErrTimeout = 1u;
+constexpr unsigned kErrRange = 2u;
 
 // One error word per device that loads the library.  Kernels OR flags into it;
 // awq_device_error() reads and clears it.

@@ -200,6 +200,10 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                 zmagic = zm | (zm << 16);
                 const uint32_t zn = 0xD000u | (z << 4) | 0x0400u;                  // fp16 -(64 + z): 2^6 * (1 + z/64)
                 zneg16 = zn | (zn << 16);
+                // the fp16 product (q - z) * scale16 is finite for every code of the group
+                // iff max|q - z| * scale16 < 65520 (exact in fp32); otherwise flag it
+                const float qz_max = zp ? fmaxf((float)z, 15.0f - (float)z) : 8.0f;
+                if (!(h2f((uint16_t)sc) * qz_max < 65520.0f) && !isnan(h2f((uint16_t)sc))) raise_error(kErrRange);
             }
             {   // prefetch the next k-block's group parameters if the group changes
                 const int kn = k + kGemmKB;

@@ -156,6 +156,13 @@ quantize_pack_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict_
     }
 }
 
+// A kernel with no work, enqueued right after a kernel that writes packed weights.  The
+// GEMV is launched as a programmatic dependent and streams its weights before it waits
+// for the previous kernel on the stream, so that previous kernel must not be the one
+// that wrote them; this one is launched with an ordinary stream dependency, so it
+// starts only after the writer has completed and its stores are visible.
+__global__ void stream_order_kernel() {}
+
 // Column sums of |X| in fp64.  Every partial sum is an exact fp64 number (fp16
 // values are multiples of 2^-24 and the sums stay far below 2^29), so the atomic
 // accumulation is exact and order-independent.  Block: 128 threads x 8 columns;

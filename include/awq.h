@@ -37,7 +37,8 @@
  *           AWQ_ERR_WORKSPACE.  A failed launch returns AWQ_ERR_CUDA.  Device-side
  *           waits are bounded: a wait that runs out sets a device error word
  *           and the kernel returns; awq_device_error() reports it as
- *           AWQ_ERR_TIMEOUT.  NaN or Inf in W or X propagate into the outputs.
+ *           AWQ_ERR_TIMEOUT (or AWQ_ERR_RANGE for the fp16 limit of
+ *           awq_linear_gemm).  NaN or Inf in W or X propagate into the outputs.
  */
 #ifndef AWQ_B200_H
 #define AWQ_B200_H
@@ -63,7 +64,9 @@ typedef enum awq_status {
     AWQ_ERR_UNSUPPORTED = 2,   /* valid but not handled (w_bit != 4, group size, M too large for GEMV) */
     AWQ_ERR_WORKSPACE = 3,     /* ws too small (see awq_workspace_bytes) */
     AWQ_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed */
-    AWQ_ERR_TIMEOUT = 5        /* a bounded device wait ran out (see awq_device_error) */
+    AWQ_ERR_TIMEOUT = 5,       /* a bounded device wait ran out (see awq_device_error) */
+    AWQ_ERR_RANGE = 6          /* awq_linear_gemm met a group whose fp16 dequantised weights
+                                  overflow (see awq_linear_gemm; reported by awq_device_error) */
 } awq_status;
 
 /* Operation ids for awq_workspace_bytes. */
@@ -92,7 +95,8 @@ int32_t awq_abi_version(void);
  *                 q     = clamp(rint(ws/scale16), -8, 7) + 8
  * ws = fp32(W)*fp32(s) is exact.  s may be NULL (s = 1: plain round-to-nearest).
  * W [N][K], s [K] -> qweight [N][K/8], scales [N][K/G], qzeros (zero_point=1 only).
- * Needs no workspace.  N, K > 0.
+ * Needs no workspace.  N, K > 0.  Ends with an ordering kernel on `stream`, so an
+ * awq_linear_gemv may directly follow it (see the ordering note there).
  */
 awq_status awq_quantize_pack(const uint16_t* W, const uint16_t* s, int32_t N, int32_t K,
                              awq_quant_config cfg, uint32_t* qweight, uint16_t* scales,
@@ -131,8 +135,16 @@ awq_status awq_fold_inverse_scale(const uint16_t* X, const uint16_t* s, int32_t 
  * Fused dequantising linear, single-token / small-batch form ("GEMV", the pages'
  * WQLinear_GEMV: batch 1 decode).  Y[m][n] = fp16( sum_k X[m][k] *
  * (q[n][k] - zero[n][k/G]) * scale16[n][k/G] ), products exact, fp32 accumulation.
- * 1 <= M <= 8 (memory-bound for M <= 2; larger batches belong to awq_linear_gemm).
+ * 1 <= M <= 8: the batch is the n = 8 side of the m16n8k16 tensor-core fragment the
+ * kernel multiplies with, so M up to 8 costs the same weight traffic as M = 1; larger
+ * batches belong to awq_linear_gemm (M > 8 returns AWQ_ERR_UNSUPPORTED).
  * Needs no workspace (ws may be NULL).
+ * Ordering: the kernel is launched as a programmatic dependent of the previous kernel
+ * on `stream` and starts streaming qweight/scales/qzeros before that kernel has
+ * completed; it reads X only after it.  So the kernel immediately before it on the
+ * stream must not write the weights.  awq_quantize_pack ends with an ordering kernel
+ * of its own, so a GEMV may follow it directly; any other writer of the weights must
+ * be followed by some other stream work (a kernel, a copy, an event wait) first.
  */
 awq_status awq_linear_gemv(const uint16_t* X, int32_t M, const uint32_t* qweight,
                            const uint16_t* scales, const uint32_t* qzeros, int32_t N, int32_t K,
@@ -145,6 +157,12 @@ awq_status awq_linear_gemv(const uint16_t* X, int32_t M, const uint32_t* qweight
  * awq_linear_gemv; the weight tile is dequantised to fp16 ((q-zero)*scale16,
  * one rounding) in shared memory and multiplied on the tcgen05 tensor cores with
  * fp32 accumulation in tensor memory.  Any M >= 1.  Needs no workspace.
+ * Range: each dequantised weight is rounded once to fp16, so it must be finite there:
+ * max|q - zero| * scale16 < 65520 for every group (max|q - zero| is max(zero, 15 - zero),
+ * or 8 without zero point).  awq_quantize_pack gives that whenever the group's scaled
+ * weights stay within about +-61000.  A group beyond it sets the device error word and
+ * the next awq_device_error() returns AWQ_ERR_RANGE (Y is then not meaningful);
+ * awq_linear_gemv has no such limit (it applies scales in fp32).
  */
 awq_status awq_linear_gemm(const uint16_t* X, int32_t M, const uint32_t* qweight,
                            const uint16_t* scales, const uint32_t* qzeros, int32_t N, int32_t K,
@@ -179,7 +197,11 @@ size_t awq_workspace_bytes(int32_t op, int32_t M, int32_t N, int32_t K, awq_quan
 /*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device: AWQ_ERR_TIMEOUT if a bounded device wait ran out since the
- * last call, AWQ_ERR_CUDA if the synchronisation itself failed, else AWQ_OK.
+ * last call, else AWQ_ERR_RANGE if awq_linear_gemm met a group outside its fp16
+ * range, AWQ_ERR_CUDA if the synchronisation itself failed, else AWQ_OK.
+ * The library keeps per-device state (launch plans, tensor maps, the address of the
+ * fixed scratch array): after cudaDeviceReset on a device, reload the library
+ * before calling it again on that device.
  */
 awq_status awq_device_error(void* stream);
 

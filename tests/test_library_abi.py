@@ -38,11 +38,11 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         s = lib.awq_status_string(code).decode()
         assert s.startswith("AWQ_")
     assert lib.awq_status_string(99).decode() == "AWQ_ERR_UNKNOWN"
-    assert lib.awq_abi_version() == 1
+    assert lib.awq_abi_version() == 2
 
 
 def _cfg(g=128, zp=1, bits=4):

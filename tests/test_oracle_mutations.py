@@ -37,6 +37,7 @@ MUTATIONS = [
     ("loss_sign", "dW = deq / s[None, :] - np.asarray(W16, dtype=np.float16).astype(np.float64)",
      "dW = deq / s[None, :] + np.asarray(W16, dtype=np.float16).astype(np.float64)"),
     ("argmax", "best = int(np.argmin(losses))", "best = int(np.argmax(losses))"),
+    ("argmin_last", "best = int(np.argmin(losses))", "best = int(len(losses) - 1 - np.argmin(losses[::-1]))"),
     ("fold_multiply", "return fp16_rn(X / s[None, :])", "return fp16_rn(X * s[None, :])"),
     ("fp16_via_f32", "return np.asarray(x).astype(np.float16)",
      "return np.asarray(x).astype(np.float32).astype(np.float16)"),

@@ -401,3 +401,17 @@ def test_scale_search_properties():
         assert all(np.array_equal(x, y) for x, y in zip(a, b) if x is not None)
     # outlier channels make scaling pay off: the search should pick alpha > 0
     assert best > 0
+
+
+def test_scale_search_ties_go_to_the_smaller_alpha():
+    """An exact tie: with |X| = 1 everywhere, m_k = 1 and s = pow(1, alpha) = 1 for every
+    alpha, so every alpha quantises the same weights the same way and all losses are the
+    same number.  The search must then return the first index (alpha = 0)."""
+    g = np.random.Generator(np.random.PCG64(85))
+    X = np.where(g.random((8, 128)) < 0.5, -1.0, 1.0).astype(np.float16)
+    W = inputs.weights(8, 128, seed=86)
+    for zp in (True, False):
+        best, alpha, s, losses = O.scale_search(X, W, 32, zp, n_grid=20)
+        assert np.all(losses == losses[0]) and losses[0] > 0
+        assert best == 0 and alpha == 0.0
+        assert np.all(s.astype(np.float32) == 1.0)
