@@ -101,26 +101,24 @@ def scales_for_alpha(m: np.ndarray, alpha: float) -> np.ndarray:
 # Group quantisation (steps a6-a7)
 # ----------------------------------------------------------------------------
 
-def quantize_groups(W16: np.ndarray, s16, G: int, zero_point: bool):
-    """Group-wise 4-bit quantisation of ws = W * diag(s).
-
-    Returns (codes [N][K] uint8 in 0..15, scale16 [N][ng] float16,
-    zeros [N][ng] uint8).  With zero_point off the zeros are the implicit 8.
-    All arithmetic is IEEE float32 (numpy float32 ops, no fused multiply-add),
-    rint is round-half-even.
-    """
+def scaled_weights(W16: np.ndarray, s16) -> np.ndarray:
+    """ws = fp32(W) * fp32(s) per input channel (exact, reading R3); s None means 1."""
     W16 = np.asarray(W16, dtype=np.float16)
-    N, K = W16.shape
-    if K % G:
-        raise ValueError("K must be a multiple of the group size")
-    ng = K // G
     w32 = W16.astype(np.float32)
     if s16 is not None:
         s32 = np.asarray(s16, dtype=np.float16).astype(np.float32)
         ws = w32 * s32[None, :]                         # exact (R3)
     else:
         ws = w32
-    g = ws.reshape(N, ng, G)
+    return ws
+
+
+def quantize_scaled_groups(g: np.ndarray, zero_point: bool):
+    """The group quantiser on scaled weights grouped as [N][ng][G] float32: returns
+    (q [N][ng][G] float32 codes 0..15, scale16 [N][ng] float16, zero [N][ng] float32).
+    All arithmetic is IEEE float32 (numpy float32 ops, no fused multiply-add), rint is
+    round-half-even."""
+    N, ng, _ = g.shape
     if zero_point:
         mx = g.max(axis=2)
         mn = g.min(axis=2)
@@ -138,6 +136,22 @@ def quantize_groups(W16: np.ndarray, s16, G: int, zero_point: bool):
         sc = scale16.astype(np.float32)
         q = np.clip(np.rint(g / sc[:, :, None]), -8, 7) + 8   # R6
         zero = np.full((N, ng), 8, dtype=np.float32)
+    return q, scale16, zero
+
+
+def quantize_groups(W16: np.ndarray, s16, G: int, zero_point: bool):
+    """Group-wise 4-bit quantisation of ws = W * diag(s).
+
+    Returns (codes [N][K] uint8 in 0..15, scale16 [N][ng] float16,
+    zeros [N][ng] uint8).  With zero_point off the zeros are the implicit 8.
+    """
+    W16 = np.asarray(W16, dtype=np.float16)
+    N, K = W16.shape
+    if K % G:
+        raise ValueError("K must be a multiple of the group size")
+    ng = K // G
+    g = scaled_weights(W16, s16).reshape(N, ng, G)
+    q, scale16, zero = quantize_scaled_groups(g, zero_point)
     codes = q.reshape(N, K).astype(np.uint8)
     return codes, scale16, zero.astype(np.uint8)
 
@@ -248,3 +262,105 @@ def scale_search(X16, W16, G: int, zero_point: bool, n_grid: int = 20):
         losses[i] = search_loss(X16, W16, scales_for_alpha(m, a), G, zero_point)
     best = int(np.argmin(losses))           # first minimum: ties go to the smaller alpha
     return best, float(alphas[best]), scales_for_alpha(m, alphas[best]), losses
+
+
+# ----------------------------------------------------------------------------
+# duo_scaling: the scale from an activation and a weight statistic (reading D1)
+# ----------------------------------------------------------------------------
+
+S_MAX = 65504.0
+
+
+def weight_absmean(W16) -> np.ndarray:
+    """w_k = (sum_n |W[n, k]|) / N in fp64: the weights' counterpart of act_absmean (the
+    sums are exact while N * max|W| < 2^29)."""
+    Wa = np.abs(np.asarray(W16, dtype=np.float16).astype(np.float64))
+    return Wa.sum(axis=0) / np.float64(Wa.shape[0])
+
+
+def duo_scales_for_alpha(m: np.ndarray, w: np.ndarray, alpha: float) -> np.ndarray:
+    """s_k = fp16_rn(min(max(a_k / b_k, 2^-14), 65504)) with a_k = max(pow(m_k, alpha), 2^-14)
+    and b_k = max(pow(w_k, 1 - alpha), 2^-14), all in fp64, rounded once to fp16.
+
+    The activation statistic raised to alpha, divided by the weight statistic raised to
+    1 - alpha (the weights' share of the scaling).  With w = 1 it is scales_for_alpha."""
+    a = np.maximum(np.power(np.asarray(m, dtype=np.float64), np.float64(alpha)), S_MIN)
+    b = np.maximum(np.power(np.asarray(w, dtype=np.float64), np.float64(1.0) - np.float64(alpha)), S_MIN)
+    return fp16_rn(np.minimum(np.maximum(a / b, S_MIN), S_MAX))
+
+
+def scale_search_duo(X16, W16, G: int, zero_point: bool, n_grid: int = 20):
+    """The grid search with duo scaling: (best_index, alpha*, s* fp16 [K], losses [n_grid]),
+    the loss and the tie rule as in scale_search."""
+    m = act_absmean(X16)
+    w = weight_absmean(W16)
+    alphas = alpha_grid(n_grid)
+    losses = np.empty(n_grid, dtype=np.float64)
+    for i, a in enumerate(alphas):
+        losses[i] = search_loss(X16, W16, duo_scales_for_alpha(m, w, a), G, zero_point)
+    top = int(np.argmin(losses))            # first minimum: ties go to the smaller alpha
+    return top, float(alphas[top]), duo_scales_for_alpha(m, w, alphas[top]), losses
+
+
+# ----------------------------------------------------------------------------
+# apply_clip: per-group weight clipping chosen by the group's output error (reading C1)
+# ----------------------------------------------------------------------------
+
+def clip_ratios(n_grid: int, n_clip: int) -> np.ndarray:
+    """r_j = 1 - j / n_grid for j = 0 .. n_clip - 1, evaluated in fp64, rounded to fp32."""
+    j = np.arange(n_clip, dtype=np.float64)
+    return (np.float64(1.0) - j / np.float64(n_grid)).astype(np.float32)
+
+
+def clip_groups(g: np.ndarray, ratio) -> np.ndarray:
+    """Clamp each group of scaled weights [N][ng][G] to [-c, c] with c = fl32(ratio *
+    max|group|); `ratio` is a float32 scalar or an [N][ng] array."""
+    amax = np.abs(g).max(axis=2)
+    c = (np.asarray(ratio, dtype=np.float32) * amax).astype(np.float32)
+    return np.clip(g, -c[:, :, None], c[:, :, None])
+
+
+def clip_errors(X16, W16, s16, G: int, zero_point: bool, n_grid: int = 20, n_clip: int = 10) -> np.ndarray:
+    """err[n, g, j] = sum_t (sum_{k in g} X[t, k] (Q(clip_j(W s)) / s - W)[n, k])^2 in fp64:
+    the objective's share of one group of one output channel, for clip ratio r_j."""
+    W16 = np.asarray(W16, dtype=np.float16)
+    N, K = W16.shape
+    ng = K // G
+    X = np.asarray(X16, dtype=np.float16).astype(np.float64)
+    Wd = W16.astype(np.float64)
+    s = np.asarray(s16, dtype=np.float16).astype(np.float64)
+    g = scaled_weights(W16, s16).reshape(N, ng, G)
+    err = np.empty((N, ng, n_clip), dtype=np.float64)
+    for j, r in enumerate(clip_ratios(n_grid, n_clip)):
+        q, scale16, zero = quantize_scaled_groups(clip_groups(g, r), zero_point)
+        deq = ((q.astype(np.float64) - zero.astype(np.float64)[:, :, None])
+               * scale16.astype(np.float64)[:, :, None]).reshape(N, K)
+        dW = deq / s[None, :] - Wd
+        for gi in range(ng):
+            E = X[:, gi * G:(gi + 1) * G] @ dW[:, gi * G:(gi + 1) * G].T      # [M][N]
+            err[:, gi, j] = (E * E).sum(axis=0)
+    return err
+
+
+def quantize_pack_clipped(W16, s16, G: int, zero_point: bool, clip_index, n_grid: int = 20):
+    """awq_quantize_pack of W * diag(s) with group (n, g) first clipped at ratio
+    r_{clip_index[n, g]}: (qweight, scales, qzeros or None)."""
+    W16 = np.asarray(W16, dtype=np.float16)
+    N, K = W16.shape
+    ng = K // G
+    idx = np.asarray(clip_index)
+    ratios = clip_ratios(n_grid, int(idx.max()) + 1)[idx]
+    g = clip_groups(scaled_weights(W16, s16).reshape(N, ng, G), ratios)
+    q, scale16, zero = quantize_scaled_groups(g, zero_point)
+    qweight = pack_nibbles(q.reshape(N, K).astype(np.uint8))
+    qzeros = pack_nibbles(zero.astype(np.uint8)) if zero_point else None
+    return qweight, scale16, qzeros
+
+
+def clip_search(X16, W16, s16, G: int, zero_point: bool, n_grid: int = 20, n_clip: int = 10):
+    """apply_clip: per (n, g) the clip index with the smallest error (ties to the smaller
+    index, i.e. less clipping), and the packed weights clipped accordingly:
+    (clip_index [N][ng] int, err [N][ng][n_clip], (qweight, scales, qzeros))."""
+    err = clip_errors(X16, W16, s16, G, zero_point, n_grid, n_clip)
+    idx = np.argmin(err, axis=2)            # first minimum
+    return idx, err, quantize_pack_clipped(W16, s16, G, zero_point, idx, n_grid)

@@ -41,6 +41,19 @@ MUTATIONS = [
     ("fold_multiply", "return fp16_rn(X / s[None, :])", "return fp16_rn(X * s[None, :])"),
     ("fp16_via_f32", "return np.asarray(x).astype(np.float16)",
      "return np.asarray(x).astype(np.float32).astype(np.float16)"),
+    ("wmean_no_abs", "Wa = np.abs(np.asarray(W16", "Wa = (np.asarray(W16"),
+    ("duo_weight_exponent_alpha", "np.float64(1.0) - np.float64(alpha)", "np.float64(alpha)"),
+    ("duo_multiply", "np.minimum(np.maximum(a / b, S_MIN), S_MAX)", "np.minimum(np.maximum(a * b, S_MIN), S_MAX)"),
+    ("duo_no_cap", "np.minimum(np.maximum(a / b, S_MIN), S_MAX)", "np.maximum(a / b, S_MIN)"),
+    ("duo_argmax", "top = int(np.argmin(losses))", "top = int(np.argmax(losses))"),
+    ("clip_ratio_sign", "np.float64(1.0) - j / np.float64(n_grid)", "np.float64(1.0) + j / np.float64(n_grid)"),
+    ("clip_no_fp32_ratio", "c = (np.asarray(ratio, dtype=np.float32) * amax).astype(np.float32)",
+     "c = (np.asarray(ratio, dtype=np.float64) * 0.999 * amax).astype(np.float32)"),
+    ("clip_reference_clipped", "dW = deq / s[None, :] - Wd",
+     "dW = deq / s[None, :] - (clip_groups(g, r).reshape(N, K) / s[None, :])"),
+    ("clip_argmax", "idx = np.argmin(err, axis=2)", "idx = np.argmax(err, axis=2)"),
+    ("clip_group_transposed", "E = X[:, gi * G:(gi + 1) * G] @ dW[:, gi * G:(gi + 1) * G].T",
+     "E = X[:, gi * G:(gi + 1) * G] @ dW[:, gi * G:(gi + 1) * G][:, ::-1].T"),
 ]
 
 PIN_NAMES = [n for n in dir(P) if n.startswith("test_")]

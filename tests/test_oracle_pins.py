@@ -415,3 +415,195 @@ def test_scale_search_ties_go_to_the_smaller_alpha():
         assert np.all(losses == losses[0]) and losses[0] > 0
         assert best == 0 and alpha == 0.0
         assert np.all(s.astype(np.float32) == 1.0)
+
+
+# ----------------------------------------------------------------------------
+# duo_scaling
+# ----------------------------------------------------------------------------
+
+def exact_round_fp16_q(q: Fraction) -> float:
+    """exact_round_fp16 for an exact rational."""
+    import bisect
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    if a >= _FP16_OVERFLOW:
+        return sign * math.inf
+    i = bisect.bisect_left(_FP16_VALUES, a)
+    if i < len(_FP16_VALUES) and _FP16_VALUES[i] == a:
+        return sign * float(a)
+    lo_v, lo_b = _FP16[i - 1]
+    hi_v, hi_b = _FP16[i] if i < len(_FP16) else (Fraction(65536), 0x7C00)
+    d_lo, d_hi = a - lo_v, hi_v - a
+    if d_lo < d_hi or (d_lo == d_hi and lo_b % 2 == 0):
+        return sign * float(lo_v)
+    return sign * float(hi_v)
+
+
+def test_weight_absmean_is_the_exact_mean():
+    W = inputs.weights(37, 24, 0.3, seed=90)
+    got = O.weight_absmean(W)
+    for k in range(24):
+        want = sum(abs(Fraction(float(v))) for v in W[:, k]) / 37
+        assert got[k] == float(want)
+
+
+def test_duo_scales_closed_form():
+    """s = fp16(min(max(a / b, 2^-14), 65504)), a = max(m^alpha, 2^-14), b = max(w^(1-alpha),
+    2^-14), against 40-digit decimal arithmetic rounded exactly to fp16 (cases within 1e-12 of
+    an fp16 midpoint are skipped); includes the clamps (tiny w, zero m)."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 40
+    g = np.random.Generator(np.random.PCG64(91))
+    m = np.concatenate([g.uniform(0.05, 30.0, 40), [0.0, 3.0, 1e-7, 30.0]])
+    w = np.concatenate([g.uniform(1e-3, 0.5, 40), [0.02, 1e-12, 0.01, 1e-12]])
+    checked = 0
+    for alpha in (0.0, 0.05, 0.35, 0.5, 0.95):
+        got = O.duo_scales_for_alpha(m, w, alpha).astype(np.float64)
+        lo = Decimal(2) ** -14
+        for k in range(len(m)):
+            al = Decimal(float(np.float64(alpha)))
+            a = Decimal(float(m[k])) ** al if m[k] > 0 else (Decimal(1) if alpha == 0 else Decimal(0))
+            b = Decimal(float(w[k])) ** (1 - al)
+            v = min(max(max(a, lo) / max(b, lo), lo), Decimal(65504))
+            q = Fraction(str(v))
+            want = exact_round_fp16_q(q)
+            if q != Fraction(want):             # skip values within 1e-12 of an fp16 midpoint
+                nxt = np.nextafter(np.float16(want), np.float16(np.inf)).astype(np.float64)
+                prv = np.nextafter(np.float16(want), np.float16(0)).astype(np.float64)
+                mids = [(Fraction(want) + Fraction(float(x))) / 2 for x in (nxt, prv) if np.isfinite(x)]
+                if min(abs(q - mm) for mm in mids) <= q * Fraction(1, 10 ** 12):
+                    continue
+            assert got[k] == want, (alpha, k, got[k], want)
+            checked += 1
+    assert checked > 150
+
+
+def test_duo_search_with_unit_weight_statistic_is_the_plain_search():
+    """With |W| = 1 everywhere the weight statistic is 1, and duo scaling reduces to the
+    plain search exactly: the same s for every alpha, the same losses and index."""
+    g = np.random.Generator(np.random.PCG64(92))
+    W = np.where(g.random((24, 256)) < 0.5, -1.0, 1.0).astype(np.float16)
+    X = inputs.activations(32, 256, seed=93)
+    m = O.act_absmean(X)
+    w = O.weight_absmean(W)
+    assert np.all(w == 1.0)
+    for a in O.alpha_grid(20):
+        assert np.array_equal(O.duo_scales_for_alpha(m, w, a), O.scales_for_alpha(m, a))
+    for zp in (True, False):
+        d = O.scale_search_duo(X, W, 64, zp, 20)
+        p = O.scale_search(X, W, 64, zp, 20)
+        assert d[0] == p[0] and np.array_equal(d[2], p[2]) and np.array_equal(d[3], p[3])
+
+
+def test_duo_search_properties():
+    X = inputs.activations(32, 256, seed=94)
+    W = inputs.weights(16, 256, seed=95)
+    m, w = O.act_absmean(X), O.weight_absmean(W)
+    for zp in (True, False):
+        best, alpha, s, losses = O.scale_search_duo(X, W, 64, zp, 20)
+        assert best == int(np.argmin(losses)) and losses[best] <= losses.min()
+        assert np.array_equal(s, O.duo_scales_for_alpha(m, w, alpha))
+        # every loss is the plain search's loss function at the duo s of that alpha
+        for i in (0, 7, 19):
+            assert losses[i] == O.search_loss(X, W, O.duo_scales_for_alpha(m, w, i / 20), 64, zp)
+    # alpha = 0: s = fp16(1 / w) (the weights alone set the scale)
+    s0 = O.duo_scales_for_alpha(m, w, 0.0).astype(np.float64)
+    for k in range(0, 256, 17):
+        assert s0[k] == exact_round_fp16_q(1 / Fraction(float(w[k])))
+
+
+# ----------------------------------------------------------------------------
+# apply_clip
+# ----------------------------------------------------------------------------
+
+def test_clip_ratios_closed_form():
+    r = O.clip_ratios(20, 10)
+    assert r.dtype == np.float32 and len(r) == 10
+    for j in range(10):
+        assert r[j] == np.float32(Fraction(20 - j, 20))
+
+
+def test_clip_with_one_ratio_is_plain_quantisation():
+    """n_clip = 1: the only ratio is 1 (clamping at the group's own max|ws|), so the
+    result is awq_quantize_pack of W s, bit for bit."""
+    X = inputs.activations(16, 256, seed=96)
+    W = inputs.weights(12, 256, seed=97)
+    s = O.scales_for_alpha(O.act_absmean(X), 0.5)
+    for G in (32, 128):
+        for zp in (True, False):
+            idx, err, packed = O.clip_search(X, W, s, G, zp, 20, 1)
+            assert np.all(idx == 0)
+            ref = O.quantize_pack(W, s, G, zp)
+            assert all(np.array_equal(a, b) for a, b in zip(packed, ref) if a is not None)
+
+
+def test_clip_error_of_one_group_is_the_search_loss():
+    """With K = G there is one group: sum_n err[n, 0, 0] / (M N) is the search loss."""
+    X = inputs.activations(24, 64, seed=98)
+    W = inputs.weights(10, 64, seed=99)
+    s = O.scales_for_alpha(O.act_absmean(X), 0.4)
+    for zp in (True, False):
+        err = O.clip_errors(X, W, s, 64, zp, 20, 3)
+        want = O.search_loss(X, W, s, 64, zp)
+        assert abs(err[:, 0, 0].sum() / (24 * 10) - want) <= 1e-12 * want
+
+
+def _brute_clip_err(X, W, s, G, zp, ratio):
+    """Independent per-group clip + quantise by scanning all 16 codes, then the group's
+    output error with Python sums."""
+    N, K = W.shape
+    ws = W.astype(np.float32) * s.astype(np.float32)[None, :]
+    Xd = X.astype(np.float64)
+    out = np.zeros((N, K // G))
+    for n in range(N):
+        for gi in range(K // G):
+            grp = ws[n, gi * G:(gi + 1) * G]
+            c = np.float32(np.float32(ratio) * np.float32(max(abs(float(v)) for v in grp)))
+            grp = np.array([min(max(float(v), -float(c)), float(c)) for v in grp], dtype=np.float32)
+            if zp:
+                sc32 = np.float32(np.float32(grp.max()) - np.float32(grp.min())) / np.float32(15)
+                sc = float(np.float16(max(sc32, np.float32(1e-5))))
+                z = min(max(round(float(np.float32(-grp.min()) / np.float32(sc))), 0), 15)
+            else:
+                sc32 = np.float32(np.abs(grp).max()) / np.float32(7)
+                sc = float(np.float16(max(sc32, np.float32(1e-5))))
+                z = 8
+            dw = []
+            for j, v in enumerate(grp):
+                d = [abs(float(v) - (c_ - z) * sc) for c_ in range(16)]
+                c_ = min(range(16), key=lambda cc: (d[cc], (cc - z) % 2))
+                k = gi * G + j
+                dw.append((c_ - z) * sc / float(s[k]) - float(W[n, k]))
+            e = [sum(Xd[t, gi * G + j] * dw[j] for j in range(G)) for t in range(X.shape[0])]
+            out[n, gi] = sum(v * v for v in e)
+    return out
+
+
+@pytest.mark.parametrize("zp", [True, False])
+def test_clip_errors_against_brute_force(zp):
+    X = inputs.activations(6, 64, seed=100)
+    W = inputs.weights(3, 64, seed=101)
+    W[1, :32] = np.linspace(-0.05, 0.03, 32).astype(np.float16)
+    s = O.scales_for_alpha(O.act_absmean(X), 0.3)
+    err = O.clip_errors(X, W, s, 32, zp, 20, 6)
+    for j in range(6):
+        want = _brute_clip_err(X, W, s, 32, zp, np.float32(Fraction(20 - j, 20)))
+        assert np.allclose(err[:, :, j], want, rtol=1e-9, atol=0)
+
+
+def test_clip_search_properties():
+    """The chosen ratio has the smallest error of its group (first one on ties: an all-zero
+    group has equal errors for every ratio and keeps ratio 1), and the packed result is the
+    quantisation of the group clipped at that ratio; clipping can only lower the error."""
+    X = inputs.activations(32, 256, seed=102)
+    W = inputs.weights(16, 256, seed=103)
+    W[4] = 0
+    s = O.scales_for_alpha(O.act_absmean(X), 0.5)
+    for zp in (True, False):
+        idx, err, packed = O.clip_search(X, W, s, 64, zp, 20, 10)
+        chosen = np.take_along_axis(err, idx[:, :, None], axis=2)[:, :, 0]
+        assert np.all(chosen == err.min(axis=2)) and np.all(chosen <= err[:, :, 0])
+        assert np.all(idx[4] == 0)
+        assert np.any(idx > 0)              # some group prefers clipping
+        ref = O.quantize_pack_clipped(W, s, 64, zp, idx, 20)
+        assert all(np.array_equal(a, b) for a, b in zip(packed, ref) if a is not None)
