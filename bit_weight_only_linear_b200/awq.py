@@ -40,6 +40,9 @@ SIGNATURES = {
     "awq_scale_search": (ctypes.c_int, [_u16p, ctypes.c_int32, _u16p, ctypes.c_int32, ctypes.c_int32,
                                         QuantConfig, ctypes.c_int32, _u16p, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "awq_scale_search_duo": (ctypes.c_int, [_u16p, ctypes.c_int32, _u16p, ctypes.c_int32, ctypes.c_int32,
+                                            QuantConfig, ctypes.c_int32, _u16p, ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "awq_scale_search_noalloc": (ctypes.c_int, [_u16p, ctypes.c_int32, _u16p, ctypes.c_int32, ctypes.c_int32,
                                                 QuantConfig, ctypes.c_int32, _u16p, ctypes.c_void_p,
                                                 ctypes.c_void_p, ctypes.c_void_p]),
@@ -51,6 +54,12 @@ SIGNATURES = {
     "awq_linear_gemm": (ctypes.c_int, [_u16p, ctypes.c_int32, _u32p, _u16p, _u32p, ctypes.c_int32,
                                        ctypes.c_int32, QuantConfig, _u16p, ctypes.c_void_p, ctypes.c_size_t,
                                        ctypes.c_void_p]),
+    "awq_apply_clip": (ctypes.c_int, [_u16p, ctypes.c_int32, _u16p, _u16p, ctypes.c_int32, ctypes.c_int32,
+                                      QuantConfig, ctypes.c_int32, ctypes.c_int32, _u32p, _u16p, _u32p,
+                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                      ctypes.c_void_p]),
+    "awq_apply_clip_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                         QuantConfig, ctypes.c_int32]),
     "awq_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                               QuantConfig]),
     "awq_device_error": (ctypes.c_int, [ctypes.c_void_p]),
@@ -185,35 +194,44 @@ def workspace_bytes(op: int, M: int, N: int, K: int, group_size: int = 128, zero
 
 
 def scale_search(X: torch.Tensor, W: torch.Tensor, group_size: int = 128, zero_point: bool = True,
-                 n_grid: int = 20, workspace: Optional[torch.Tensor] = None, stream=None
-                 ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """awq_scale_search: returns (s* fp16 [K], losses fp64 [n_grid], best index int32 [1]), all on device."""
+                 n_grid: int = 20, workspace: Optional[torch.Tensor] = None, stream=None, out=None,
+                 duo_scaling: bool = False) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """awq_scale_search (awq_scale_search_duo with duo_scaling): returns (s* fp16 [K], losses
+    fp64 [n_grid], best index int32 [1]), all on device (into `out` = (s, losses, best) when
+    given)."""
     M, K = X.shape
     N = W.shape[0]
-    need = workspace_bytes(AWQ_OP_SCALE_SEARCH, M, N, K, group_size, zero_point)
     if workspace is None:
+        need = workspace_bytes(AWQ_OP_SCALE_SEARCH, M, N, K, group_size, zero_point)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
-    s_out = torch.empty(K, dtype=torch.float16, device=X.device)
-    losses = torch.empty(n_grid, dtype=torch.float64, device=X.device)
-    best = torch.empty(1, dtype=torch.int32, device=X.device)
-    st = load_library().awq_scale_search(
+    if out is None:
+        s_out = torch.empty(K, dtype=torch.float16, device=X.device)
+        losses = torch.empty(n_grid, dtype=torch.float64, device=X.device)
+        best = torch.empty(1, dtype=torch.int32, device=X.device)
+    else:
+        s_out, losses, best = out
+    name = "awq_scale_search_duo" if duo_scaling else "awq_scale_search"
+    st = getattr(load_library(), name)(
         _dev(X, "X", _F16), M, _dev(W, "W", _F16), N, K, config(group_size, zero_point), n_grid,
         _dev(s_out, "s_out", _F16), losses.data_ptr(), best.data_ptr(), workspace.data_ptr(),
         workspace.numel() * workspace.element_size(), _stream(stream))
-    _check("awq_scale_search", st)
+    _check(name, st)
     return s_out, losses, best
 
 
 def scale_search_noalloc(X: torch.Tensor, W: torch.Tensor, group_size: int = 128, zero_point: bool = True,
-                         n_grid: int = 20, stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+                         n_grid: int = 20, stream=None, out=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """awq_scale_search_noalloc: the scale search on the library's fixed scratch (for
     callers that cannot allocate device memory).  Returns (s*, losses, best index) on
-    device; the output tensors here are allocated by torch only for convenience."""
+    device, into `out` when given (otherwise torch allocates them here, for convenience)."""
     M, K = X.shape
     N = W.shape[0]
-    s_out = torch.empty(K, dtype=torch.float16, device=X.device)
-    losses = torch.empty(n_grid, dtype=torch.float64, device=X.device)
-    best = torch.empty(1, dtype=torch.int32, device=X.device)
+    if out is None:
+        s_out = torch.empty(K, dtype=torch.float16, device=X.device)
+        losses = torch.empty(n_grid, dtype=torch.float64, device=X.device)
+        best = torch.empty(1, dtype=torch.int32, device=X.device)
+    else:
+        s_out, losses, best = out
     st = load_library().awq_scale_search_noalloc(
         _dev(X, "X", _F16), M, _dev(W, "W", _F16), N, K, config(group_size, zero_point), n_grid,
         _dev(s_out, "s_out", _F16), losses.data_ptr(), best.data_ptr(), _stream(stream))
@@ -230,3 +248,35 @@ def check_bounded_wait(stream=None) -> None:
 def device_error(stream=None) -> None:
     """Synchronise and raise AWQError if a bounded device wait ran out."""
     _check("awq_device_error", load_library().awq_device_error(_stream(stream)))
+
+
+def apply_clip(X: torch.Tensor, W: torch.Tensor, s: Optional[torch.Tensor], group_size: int = 128,
+               zero_point: bool = True, n_grid: int = 20, n_clip: int = 10, out=None,
+               workspace: Optional[torch.Tensor] = None, stream=None, errors: bool = False):
+    """awq_apply_clip: per-group clip ratio chosen by the group's output error, then the
+    packed clipped weights.  Returns (qweight, scales, qzeros or None, clip index uint8
+    [N][K/G]), plus the errors fp64 [N][K/G][n_clip] when `errors`."""
+    M, K = X.shape
+    N = W.shape[0]
+    lib = load_library()
+    if workspace is None:
+        need = int(lib.awq_apply_clip_workspace_bytes(M, N, K, config(group_size, zero_point), n_clip))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
+    qs, ss, zs = packed_shapes(N, K, group_size, zero_point)
+    if out is None:
+        qweight = torch.empty(qs, dtype=torch.int32, device=W.device)
+        scales = torch.empty(ss, dtype=torch.float16, device=W.device)
+        qzeros = torch.empty(zs, dtype=torch.int32, device=W.device) if zero_point else None
+        idx = torch.empty((N, K // group_size), dtype=torch.uint8, device=W.device)
+    else:
+        qweight, scales, qzeros, idx = out
+    err = torch.empty((N, K // group_size, n_clip), dtype=torch.float64, device=W.device) if errors else None
+    st = lib.awq_apply_clip(
+        _dev(X, "X", _F16), M, _dev(W, "W", _F16), _dev(s, "s", _F16), N, K, config(group_size, zero_point),
+        n_grid, n_clip, _dev(qweight, "qweight", _W32), _dev(scales, "scales", _F16), _dev(qzeros, "qzeros", _W32),
+        0 if idx is None else idx.data_ptr(), 0 if err is None else err.data_ptr(), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("awq_apply_clip", st)
+    if errors:
+        return qweight, scales, qzeros, idx, err
+    return qweight, scales, qzeros, idx

@@ -112,15 +112,61 @@ awq_status awq_quantize_pack(const uint16_t* W, const uint16_t* s, int32_t N, in
  * best alpha; losses_out [n_grid] fp64 and best_index_out [1] int32 are DEVICE
  * pointers and may be NULL.  alpha* = best_index / n_grid.
  * X [M][K] are the calibration activations (M >= 1 tokens), W [N][K].
- * 1 <= n_grid <= 64.  ws_bytes >= awq_workspace_bytes(AWQ_OP_SCALE_SEARCH, M, N, K, cfg).
- * Every fp32 product of the loss uses X exactly and Q(Ws)/s - W split into two
- * fp16 terms (22-bit significand), accumulated in fp32 on the tensor cores and
- * summed in fp64.
+ * 1 <= n_grid <= 64.  ws_bytes >= awq_workspace_bytes(AWQ_OP_SCALE_SEARCH, M, N, K, cfg)
+ * (a few MB: statistics, the s table, per-tile partial sums; Q(Ws)/s - W is built
+ * tile by tile in shared memory and never stored).
+ * Every fp32 product of the loss uses X exactly and Q(Ws)/s - W (scaled by a power of
+ * two per alpha) split into two fp16 terms (22-bit significand), accumulated in fp32
+ * on the tensor cores and summed in fp64.
+ * Results stay on the device and the call is asynchronous like the others (the host
+ * reads best_index_out when it needs alpha; nothing here synchronises the stream).
  */
 awq_status awq_scale_search(const uint16_t* X, int32_t M, const uint16_t* W, int32_t N,
                             int32_t K, awq_quant_config cfg, int32_t n_grid, uint16_t* s_out,
                             double* losses_out, int32_t* best_index_out, void* ws,
                             size_t ws_bytes, void* stream);
+
+/*
+ * The scale search with duo scaling (lshu.cn guide, 校准参数全景: duo_scaling, "scale
+ * weights and activations"): the same grid, loss, tie rule, outputs and workspace as
+ * awq_scale_search, with the scale of alpha_i taken from both statistics,
+ *   s_i = fp16(min(max(max(pow(m_k, alpha_i), 2^-14) / max(pow(w_k, 1 - alpha_i), 2^-14),
+ *                      2^-14), 65504)),   w_k = mean_n |W[n][k]| (fp64),
+ * all in fp64 with one rounding to fp16 (with w = 1 it is the plain search's s).
+ */
+awq_status awq_scale_search_duo(const uint16_t* X, int32_t M, const uint16_t* W, int32_t N,
+                                int32_t K, awq_quant_config cfg, int32_t n_grid, uint16_t* s_out,
+                                double* losses_out, int32_t* best_index_out, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/*
+ * Weight clipping chosen by the output error (lshu.cn guide, 校准参数全景: apply_clip,
+ * clip the weights to further reduce the effect of outliers on the quantisation error),
+ * then group quantisation and packing of the clipped weights.  With ws = W * diag(s)
+ * (s from the scale search; NULL = 1), for every output channel n, group g and clip ratio
+ * r_j = fl32(1 - j/n_grid), j = 0 .. n_clip-1:
+ *   c_j = fl32(r_j * max|ws| over the group),  Q_j = the quantiser of awq_quantize_pack
+ *   applied to clamp(ws, -c_j, c_j),
+ *   err_j = sum_t ( sum_{k in g} X[t][k] * (Q_j/s - W)[n][k] )^2
+ * (the objective's share of that group; X the calibration activations as given to the
+ * search).  Each group keeps the j with the smallest err_j (ties to the smaller j, i.e.
+ * less clipping) and is written into qweight/scales/qzeros clipped at it, in the layout of
+ * awq_quantize_pack; clip_index_out [N][K/G] uint8 (DEVICE, may be NULL) receives j and
+ * err_out [N][K/G][n_clip] fp64 (DEVICE, may be NULL) every err_j.
+ * 1 <= n_clip <= min(n_grid, 32).  ws_bytes >= awq_apply_clip_workspace_bytes(...).
+ * err_j is evaluated on the tensor cores: Q_j/s - W split into two fp16 terms (22-bit
+ * significand), X exact, fp32 accumulation over the group, squares summed in fp32 per 16
+ * tokens and in fp64 beyond.  Ends with an ordering kernel (see awq_linear_gemv).
+ */
+awq_status awq_apply_clip(const uint16_t* X, int32_t M, const uint16_t* W, const uint16_t* s,
+                          int32_t N, int32_t K, awq_quant_config cfg, int32_t n_grid,
+                          int32_t n_clip, uint32_t* qweight, uint16_t* scales, uint32_t* qzeros,
+                          uint8_t* clip_index_out, double* err_out, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Workspace bytes of awq_apply_clip (0 for invalid sizes). */
+size_t awq_apply_clip_workspace_bytes(int32_t M, int32_t N, int32_t K, awq_quant_config cfg,
+                                      int32_t n_clip);
 
 /*
  * Activation side of the scaling (lshu.cn guide, 算法原理: "s^-1 * X"):
@@ -137,7 +183,9 @@ awq_status awq_fold_inverse_scale(const uint16_t* X, const uint16_t* s, int32_t 
  * (q[n][k] - zero[n][k/G]) * scale16[n][k/G] ), products exact, fp32 accumulation.
  * 1 <= M <= 8: the batch is the n = 8 side of the m16n8k16 tensor-core fragment the
  * kernel multiplies with, so M up to 8 costs the same weight traffic as M = 1; larger
- * batches belong to awq_linear_gemm (M > 8 returns AWQ_ERR_UNSUPPORTED).
+ * batches belong to awq_linear_gemm (M > 8 returns AWQ_ERR_UNSUPPORTED).  The M rows
+ * of X are staged in shared memory; when M * K * 2 bytes do not fit (e.g. 8 x 14336) the
+ * batch is processed in parts, one launch each, each streaming the weights once.
  * Needs no workspace (ws may be NULL).
  * Ordering: the kernel is launched as a programmatic dependent of the previous kernel
  * on `stream` and starts streaming qweight/scales/qzeros before that kernel has

@@ -56,4 +56,16 @@ def test_traffic_record_guarded_by_the_gemv_code(monkeypatch, tmp_path):
 
 def test_gemv_sources_are_the_gemv_files():
     names = sorted(os.path.basename(p) for p in bench.gemv_sources())
-    assert names == ["awq_api.cu", "common.cuh", "gemv.cuh", "launch.cuh", "sm100.cuh"]
+    assert names == ["common.cuh", "gemv.cuh", "gemv_launch.cuh", "launch.cuh", "sm100.cuh"]
+
+
+def test_every_traffic_tag_names_existing_sources():
+    for tag, names in bench.KERNEL_SOURCES.items():
+        found = sorted(os.path.basename(p) for p in bench.kernel_sources(tag))
+        assert found == sorted(names), tag
+
+
+def test_rotations_exceed_twice_the_l2():
+    for nbytes in (8_716_288, 113_451_008, 300_000_000):
+        r = bench.rotations_for(nbytes)
+        assert r * nbytes > 2 * bench.L2_BYTES and r >= 2

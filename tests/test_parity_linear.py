@@ -9,6 +9,7 @@ import torch
 
 import inputs
 from helpers import assert_linear_close, to_dev, to_np
+from bit_weight_only_linear_b200 import awq as _awq
 from oracle import awq_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -177,5 +178,79 @@ def test_gemm_llama70b_prefill_sampled(lib):
         y = to_np(lib.linear_gemm(to_dev(X), q, sc, z, 128, True))
         lib.device_error()
         rows = np.sort(rng.choice(N, 128, replace=False))
-        ref = O.linear_rows(X, to_np(q), to_np(sc), to_np(z), K, 128, True, rows)
+        # the GPU's packing of the sampled rows, bit for bit against the oracle's
+        rq, rs, rz = O.quantize_pack(W[rows], None, 128, True)
+        assert np.array_equal(to_np(q)[rows], rq)
+        assert np.array_equal(to_np(sc)[rows].view(np.uint16), rs.view(np.uint16))
+        assert np.array_equal(to_np(z)[rows], rz)
+        ref = O.linear_rows(X, rq, rs, rz, K, 128, True, np.arange(len(rows)))
         assert_linear_close(y[:, rows], ref)
+
+
+def _edge_weights(K):
+    """Rows of constant groups (scale at the 1e-5 floor), and rows of large magnitude
+    (group ranges up to ~4e4: scale16 near 2700, the fp16 products (q - z) * scale16 up
+    to ~4e4, still finite)."""
+    g = np.random.Generator(np.random.PCG64(310))
+    rows = [np.zeros(K), np.full(K, 0.25), np.full(K, -3.0),
+            g.uniform(-20000, 20000, K), g.uniform(0, 30000, K), g.uniform(-40000, -100, K),
+            np.where(np.arange(K) % 3 == 0, 18000.0, -21000.0)]
+    return np.stack(rows).astype(np.float16)
+
+
+@pytest.mark.parametrize("G", O.GROUP_SIZES)
+@pytest.mark.parametrize("zp", [True, False])
+def test_gemm_edge_magnitudes(lib, G, zp):
+    """Constant groups and large-magnitude groups through both linear forms, against the
+    oracle; the activations are small so that the outputs stay finite in fp16."""
+    K, M = 512, 40
+    W = np.concatenate([_edge_weights(K)] * 3)
+    X = (inputs.activations(M, K, seed=311).astype(np.float32) * np.float32(1e-3)).astype(np.float16)
+    q, sc, z, dq = _packed(W, G, zp)
+    ref = O.linear(X, q, sc, z, K, G, zp)
+    y = _run(lib, "gemm", X, dq, G, zp)
+    lib.device_error()
+    assert_linear_close(y, ref)
+    assert_linear_close(_run(lib, "gemv", X[:3], dq, G, zp), ref[:3])
+
+
+def test_gemm_reports_fp16_overflow(lib):
+    """A group whose dequantised weights leave fp16 ((q - z) * scale16 = 15 * 5000) makes
+    the GEMM flag AWQ_ERR_RANGE; the next call on valid weights runs clean."""
+    N, K, G = 128, 256, 128
+    codes = np.random.Generator(np.random.PCG64(312)).integers(0, 16, size=(N, K)).astype(np.uint8)
+    codes[:, 0] = 15
+    scales = np.full((N, K // G), 0.01, dtype=np.float16)
+    scales[5, 1] = 5000.0
+    zeros = np.zeros((N, K // G), dtype=np.uint8)
+    dq = (to_dev(O.pack_nibbles(codes)), to_dev(scales), to_dev(O.pack_nibbles(zeros)))
+    X = (inputs.activations(16, K, seed=313).astype(np.float32) * np.float32(1e-3)).astype(np.float16)
+    lib.linear_gemm(to_dev(X), *dq, G, True)
+    with pytest.raises(_awq.AWQError) as err:
+        lib.device_error()
+    assert err.value.status == _awq.AWQ_ERR_RANGE
+    scales[5, 1] = 4000.0          # 15 * 4000 = 60000: finite
+    dq = (dq[0], to_dev(scales), dq[2])
+    y = _run(lib, "gemm", X, dq, G, True)
+    lib.device_error()
+    assert_linear_close(y, O.linear(X, O.pack_nibbles(codes), scales, O.pack_nibbles(zeros), K, G, True))
+
+
+def test_gemv_directly_after_quantize_pack(lib):
+    """The GEMV streams its weights before it waits for the previous kernel; a GEMV
+    enqueued right after awq_quantize_pack into the same buffers (no synchronisation in
+    between) must still see the new weights."""
+    N, K, G = 4096, 4096, 128
+    X = inputs.activations(1, K, seed=314)
+    Xd = to_dev(X)
+    W0 = to_dev(inputs.weights(N, K, 0.02, seed=315))
+    bufs = lib.quantize_pack(W0, None, G, True)
+    torch.cuda.synchronize()
+    for i in range(3):
+        W = inputs.weights(N, K, 0.02, seed=316 + i)
+        Wd = to_dev(W)
+        torch.cuda.synchronize()
+        lib.quantize_pack(Wd, None, G, True, out=bufs)
+        y = to_np(lib.linear_gemv(Xd, *bufs, G, True))
+        q, sc, z = O.quantize_pack(W, None, G, True)
+        assert_linear_close(y, O.linear(X, q, sc, z, K, G, True))

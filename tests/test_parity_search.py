@@ -18,36 +18,19 @@ import pytest
 import torch
 
 import inputs
-from helpers import to_dev, to_np
+from helpers import check_search_result, to_dev, to_np
 from oracle import awq_oracle as O
 
 pytestmark = pytest.mark.gpu
-
-LOSS_REL = 5e-5
 
 
 def _check(lib, X, W, G, zp, n_grid=20):
     s, losses, best = lib.scale_search(to_dev(X), to_dev(W), G, zp, n_grid)
     torch.cuda.synchronize()
     lib.device_error()
-    s, losses, best = to_np(s), losses.cpu().numpy(), int(best.cpu().item())
-    rb, ralpha, rs, rlosses = O.scale_search(X, W, G, zp, n_grid)
-    if best != rb:
-        assert abs(best - rb) == 1, (best, rb)
-        assert abs(rlosses[best] - rlosses[rb]) <= 1e-6 * rlosses[rb], (best, rb)
-    else:
-        diff = s.view(np.uint16) != rs.view(np.uint16)
-        if diff.any():
-            m = O.act_absmean(X)
-            p = np.power(m[diff], ralpha)
-            # allowed only where pow's value sits within 1e-12 of an fp16 midpoint
-            lo = rs[diff].astype(np.float64)
-            hi = s[diff].astype(np.float64)
-            mid = (lo + hi) / 2
-            assert np.all(np.abs(p - mid) <= 1e-12 * np.abs(mid)), "s* differs"
-    rel = np.abs(losses - rlosses) / np.maximum(rlosses, 1e-300)
-    assert rel.max() <= LOSS_REL, f"loss rel err {rel.max():.3g}"
-    return best, rb
+    got = (to_np(s), losses.cpu().numpy(), int(best.cpu().item()))
+    ref = O.scale_search(X, W, G, zp, n_grid)
+    return check_search_result(X, got, ref), ref[0]
 
 
 SMALL = [(16, 128, 8), (33, 256, 64), (64, 512, 130), (128, 1024, 256), (200, 512, 96), (40, 96, 40)]
@@ -81,9 +64,66 @@ def test_scale_search_alpha0_is_rtn(lib):
     assert np.all(to_np(s).astype(np.float32) == 1.0)
 
 
-@pytest.mark.parametrize("G,zp", [(128, True), (32, False)])
-def test_scale_search_full_layer(lib, G, zp):
-    """4096 x 4096 layer, 512 calibration tokens, 20 alphas (the quantisation sweep's size)."""
+def test_scale_search_exact_tie_picks_the_first_alpha(lib):
+    """|X| = 1 everywhere: s = 1 for every alpha, all losses are the same number on the
+    GPU as well (identical work), and the index must be 0."""
+    g = np.random.Generator(np.random.PCG64(85))
+    X = np.where(g.random((64, 512)) < 0.5, -1.0, 1.0).astype(np.float16)
+    W = inputs.weights(96, 512, seed=86)
+    for zp in (True, False):
+        s, losses, best = lib.scale_search(to_dev(X), to_dev(W), 128, zp, 20)
+        lib.device_error()
+        losses = losses.cpu().numpy()
+        assert np.all(losses == losses[0]) and int(best.cpu().item()) == 0
+        assert np.all(to_np(s).astype(np.float32) == 1.0)
+
+
+def _duo_exact(X, W):
+    m, w = O.act_absmean(X), O.weight_absmean(W)
+
+    def f(alpha):
+        a = np.maximum(np.power(m, alpha), O.S_MIN)
+        b = np.maximum(np.power(w, 1.0 - alpha), O.S_MIN)
+        return np.minimum(np.maximum(a / b, O.S_MIN), O.S_MAX)
+    return f
+
+
+def _check_duo(lib, X, W, G, zp, n_grid=20):
+    s, losses, best = lib.scale_search(to_dev(X), to_dev(W), G, zp, n_grid, duo_scaling=True)
+    lib.device_error()
+    got = (to_np(s), losses.cpu().numpy(), int(best.cpu().item()))
+    ref = O.scale_search_duo(X, W, G, zp, n_grid)
+    return check_search_result(X, got, ref, s_exact=_duo_exact(X, W))
+
+
+@pytest.mark.parametrize("G", O.GROUP_SIZES)
+@pytest.mark.parametrize("zp", [True, False])
+@pytest.mark.parametrize("mkn", [(33, 256, 64), (128, 1024, 256), (40, 96, 40)], ids=lambda t: "x".join(map(str, t)))
+def test_scale_search_duo_parity(lib, G, zp, mkn):
+    M, K, N = mkn
+    if K % G:
+        pytest.skip("K % G")
+    X = inputs.activations(M, K, seed=410 + M + K)
+    W = inputs.weights(N, K, 0.02, seed=411 + N + K)
+    _check_duo(lib, X, W, G, zp)
+
+
+def test_scale_search_duo_full_layer(lib):
+    """The quantisation sweep's layer (4096 x 4096, 512 tokens, 20 alphas), G = 128 with zero point."""
     X = inputs.activations(512, 4096, inputs.SEED_X + 40, inputs.SEED_OUTLIER + 40)
     W = inputs.weights(4096, 4096, 0.02, inputs.SEED_W + 40)
-    _check(lib, X, W, G, zp)
+    _check_duo(lib, X, W, 128, True)
+
+
+def test_scale_search_duo_with_unit_weights_is_the_plain_search(lib):
+    """|W| = 1: the weight statistic is 1, every s equals the plain search's, and so does
+    every loss, bit for bit (the same work on the same inputs)."""
+    g = np.random.Generator(np.random.PCG64(412))
+    W = to_dev(np.where(g.random((96, 512)) < 0.5, -1.0, 1.0).astype(np.float16))
+    X = to_dev(inputs.activations(64, 512, seed=413))
+    a = lib.scale_search(X, W, 64, True, 20)
+    b = lib.scale_search(X, W, 64, True, 20, duo_scaling=True)
+    lib.device_error()
+    assert np.array_equal(to_np(a[0]).view(np.uint16), to_np(b[0]).view(np.uint16))
+    assert np.array_equal(a[1].cpu().numpy(), b[1].cpu().numpy())
+    assert int(a[2].item()) == int(b[2].item())

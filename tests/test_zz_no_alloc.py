@@ -48,19 +48,30 @@ def test_noalloc_matches_workspace_search(M, K, N, G, zp):
     W = to_dev(inputs.weights(N, K, 0.02, seed=501 + K))
     ref = awq.scale_search(X, W, G, zp, 20)
     torch.cuda.synchronize()
-    for _ in range(2):
-        got = awq.scale_search_noalloc(X, W, G, zp, 20)
+    out = (torch.empty(K, dtype=torch.float16, device="cuda"), torch.empty(20, dtype=torch.float64, device="cuda"),
+           torch.empty(1, dtype=torch.int32, device="cuda"))
+    for i in range(2):
+        if i == 1:
+            # the first call has loaded the module and looked up the array's address: from
+            # here on nothing may be allocated, by the library or on its behalf
+            free0, reserved0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_reserved()
+        got = awq.scale_search_noalloc(X, W, G, zp, 20, out=out)
         torch.cuda.synchronize()
         awq.device_error()
+        if i == 1:
+            assert torch.cuda.mem_get_info()[0] == free0 and torch.cuda.memory_reserved() == reserved0
         _compare(ref, got)
 
 
 def test_noalloc_rejects_sizes_beyond_the_fixed_scratch():
-    """K above 16384 is refused on the host, before anything is launched."""
+    """K above 16384 or M above 2^20 is refused on the host, before anything is launched
+    (the pointers below are never dereferenced)."""
     from bit_weight_only_linear_b200 import awq, build
     build.build()
     lib = awq.load_library()
     fake = 0x10000
     cfg = awq.config(128, True)
-    assert lib.awq_scale_search_noalloc(fake, 16, fake, 64, 16384 + 128, cfg, 20, fake, 0, 0, None) == 2
-    assert lib.awq_scale_search_noalloc(fake, 16, fake, 64, 256, cfg, 0, fake, 0, 0, None) == 1
+    f = lib.awq_scale_search_noalloc
+    assert f(fake, 16, fake, 64, 16384 + 128, cfg, 20, fake, 0, 0, None) == awq.AWQ_ERR_UNSUPPORTED
+    assert f(fake, (1 << 20) + 1, fake, 64, 256, cfg, 20, fake, 0, 0, None) == awq.AWQ_ERR_UNSUPPORTED
+    assert f(fake, 16, fake, 64, 256, cfg, 0, fake, 0, 0, None) == awq.AWQ_ERR_INVALID_ARG
