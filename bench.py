@@ -90,7 +90,7 @@ def read_peaks():
 KERNEL_SOURCES = {
     # tag: the files whose code defines the kernel and its launch configuration
     "gemv_mistral7b_layer": ("gemv.cuh", "gemv_launch.cuh", "sm100.cuh", "common.cuh", "launch.cuh"),
-    "gemm_llama70b_prefill": ("gemm_sm100.cuh", "sm100.cuh", "common.cuh"),
+    "gemm_llama70b_o_proj": ("gemm_sm100.cuh", "sm100.cuh", "common.cuh"),
     "quantize_pack_4096": ("quantize.cuh", "common.cuh"),
     "search_fused_4096": ("search.cuh", "quantize.cuh", "gemm_sm100.cuh", "sm100.cuh", "common.cuh"),
     "apply_clip_4096": ("clip.cuh", "search.cuh", "quantize.cuh", "gemm_sm100.cuh", "sm100.cuh", "common.cuh"),
@@ -747,13 +747,15 @@ def run_ours(args):
         extra["single_gemv"] = measure_single_gemv(awq, torch, peaks)
         extra["batched"] = measure_batched(awq, torch, peaks)
         extra["gemm"] = measure_gemm(awq, torch, peaks)
-        extra["gemm"]["traffic"] = profile_traffic("gemm_llama70b_prefill")
+        # DRAM bytes of one launch of the o_proj-shaped linear (the captured case)
+        extra["gemm"]["traffic_o_proj"] = profile_traffic("gemm_llama70b_o_proj")
         extra["quantize"] = measure_quantize(awq, torch, peaks)
         extra["quantize"]["traffic"] = profile_traffic("quantize_pack_4096")
         extra["scale_search"], _ = measure_search(awq, torch, peaks)
         extra["scale_search"]["traffic"] = profile_traffic("search_fused_4096")
         extra["scale_search_duo"], _ = measure_search(awq, torch, peaks, duo=True)
         extra["apply_clip"] = measure_clip(awq, torch, peaks)
+        extra["apply_clip"]["traffic"] = profile_traffic("apply_clip_4096")
         extra["sweep"] = measure_sweep(awq, torch, peaks)
 
     cpu = None
@@ -848,6 +850,7 @@ def run_profile(args):
       gemv      two passes of the fused decode layer (four GEMV launches each)
       gemm      one launch of each of the four Llama-70B prefill GEMMs
       gemm_small one 2048 x 8192 x 8192 GEMM (a capture-sized case)
+      gemm_m16  two 16 x 4096 x 4096 GEMMs (batched-decode size)
       quantize  three quantise/pack launches on the 4096x4096 layer
       search    two scale searches on the 4096x4096 layer with 512 tokens (G=128, zp)
       clip      two apply_clip calls on that layer (G=128, zp, 10 ratios)"""
@@ -875,6 +878,13 @@ def run_profile(args):
             awq.linear_gemm(X, q, sc, z, G, ZP)
             torch.cuda.synchronize()
             del q, sc, z, X
+    if "gemm_m16" in what:
+        W = torch.from_numpy(inputs.weights(4096, 4096, 0.02, inputs.SEED_W + 33)).cuda()
+        q, sc, z = awq.quantize_pack(W, None, G, ZP)
+        X = torch.from_numpy(inputs.activations(16, 4096, inputs.SEED_X + 33)).cuda()
+        for _ in range(2):
+            awq.linear_gemm(X, q, sc, z, G, ZP)
+        torch.cuda.synchronize()
     if "gemm_small" in what:
         W = torch.from_numpy(inputs.weights(8192, 8192, 0.015, inputs.SEED_W + 31)).cuda()
         q, sc, z = awq.quantize_pack(W, None, G, ZP)
