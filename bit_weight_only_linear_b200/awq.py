@@ -183,9 +183,30 @@ def linear_gemv(X, qweight, scales, qzeros, group_size=128, zero_point=True, out
     return _linear("awq_linear_gemv", X, qweight, scales, qzeros, group_size, zero_point, out, workspace, stream)
 
 
+_GEMM_WS = {}
+
+
+def gemm_workspace(M: int, N: int, K: int, group_size: int = 128, zero_point: bool = True, device=None):
+    """A device workspace large enough for awq_linear_gemm at these sizes (the split-K
+    partial sums), cached per device and grown on demand; None when none is needed."""
+    need = workspace_bytes(AWQ_OP_GEMM, M, N, K, group_size, zero_point)
+    if need == 0:
+        return None
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    ws = _GEMM_WS.get(dev)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        _GEMM_WS[dev] = ws
+    return ws
+
+
 def linear_gemm(X, qweight, scales, qzeros, group_size=128, zero_point=True, out=None, workspace=None,
                 stream=None) -> torch.Tensor:
-    """awq_linear_gemm: Y [M][N] = X [M][K] . deq(W)^T, tcgen05 tensor-core form (any M)."""
+    """awq_linear_gemm: Y [M][N] = X [M][K] . deq(W)^T, tcgen05 tensor-core form (any M).  A
+    batch too small to fill the GPU splits K over a workspace (the cached one of
+    gemm_workspace() unless one is given)."""
+    if workspace is None:
+        workspace = gemm_workspace(X.shape[0], qweight.shape[0], X.shape[1], group_size, zero_point, X.device)
     return _linear("awq_linear_gemm", X, qweight, scales, qzeros, group_size, zero_point, out, workspace, stream)
 
 

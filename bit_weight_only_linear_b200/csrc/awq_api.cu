@@ -163,18 +163,21 @@ awq_status awq_linear_gemv(const uint16_t* X, int32_t M, const uint32_t* qweight
 awq_status awq_linear_gemm(const uint16_t* X, int32_t M, const uint32_t* qweight, const uint16_t* scales,
                            const uint32_t* qzeros, int32_t N, int32_t K, awq_quant_config cfg, uint16_t* Y,
                            void* ws, size_t ws_bytes, void* stream) {
-    (void)ws;
-    (void)ws_bytes;
     awq_status st = check_linear(X, M, qweight, scales, qzeros, N, K, cfg, Y);
     if (st != AWQ_OK) return st;
     DeviceInfo d;
     if (!device_info(d)) return AWQ_ERR_CUDA;
+    if (ws && !aligned16(ws)) return AWQ_ERR_INVALID_ARG;
     return launch_gemm_w4a16(X, M, qweight, scales, qzeros, N, K, cfg.q_group_size, cfg.zero_point, Y,
-                             (cudaStream_t)stream, d.sms);
+                             (cudaStream_t)stream, d.sms, ws, ws ? ws_bytes : 0);
 }
 
 size_t awq_workspace_bytes(int32_t op, int32_t M, int32_t N, int32_t K, awq_quant_config cfg) {
     if (op == AWQ_OP_SCALE_SEARCH) return search_workspace_bytes(M, N, K, cfg.q_group_size, 64);
+    if (op == AWQ_OP_GEMM) {
+        DeviceInfo d;
+        return gemm_workspace_bytes(M, N, K, device_info(d) ? d.sms : 148);
+    }
     return 0;
 }
 

@@ -23,6 +23,7 @@
 // drains what it issued, frees TMEM and returns.
 #pragma once
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -84,7 +85,7 @@ template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
                   const uint16_t* __restrict__ scales, const uint32_t* __restrict__ qzeros, int M, int N, int K,
-                  int G, int zero_point, uint16_t* __restrict__ Y) {
+                  int G, int zero_point, uint16_t* __restrict__ Y, int kb_per, float* __restrict__ part) {
     using C = GemmCfg<BN>;
     using namespace sm100;
     extern __shared__ uint8_t smem_raw[];
@@ -101,7 +102,10 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
     const int lane = threadIdx.x & 31;
     const int m0 = blockIdx.x * BN;
     const int n0 = blockIdx.y * kGemmTileN;
-    const int num_kb = ceil_div(K, kGemmKB);
+    // split K: this CTA takes k-blocks [kb0, kb0 + num_kb); with part != NULL it writes
+    // fp32 partial sums to part[blockIdx.z][M][N] instead of Y
+    const int kb0 = blockIdx.z * kb_per;
+    const int num_kb = max(0, min(kb_per, ceil_div(K, kGemmKB) - kb0));
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -136,8 +140,8 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                 if (kb >= C::kStages) ok = mbar_wait(&empty[s], ((kb / C::kStages) - 1) & 1);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&full[s], C::kXBytes + C::kWBytes);
-                tma_load_2d(smem + C::kXOff + s * C::kXBytes, &tmap_x, &full[s], kb * kGemmKB, m0);
-                tma_load_2d(smem + C::kWOff + s * C::kWBytes, &tmap_q, &full[s], kb * (kGemmKB / 8), n0);
+                tma_load_2d(smem + C::kXOff + s * C::kXBytes, &tmap_x, &full[s], (kb0 + kb) * kGemmKB, m0);
+                tma_load_2d(smem + C::kWOff + s * C::kWBytes, &tmap_q, &full[s], (kb0 + kb) * (kGemmKB / 8), n0);
                 ++issued;
             }
             // Drain: every issued copy must land before the CTA may exit.
@@ -180,7 +184,7 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         const uint32_t* zrow = qzeros + (size_t)(row_ok ? n : 0) * nzw;
         // scale and zero word of the thread's group, loaded one k-block ahead (raw; using a
         // loaded value stalls on its load) and only when the group changes
-        int g_next = (kq * 16) / G;
+        int g_next = (kb0 * kGemmKB + kq * 16) / G;
         uint32_t sc_next = row_ok ? __ldg(srow + g_next) : 0u;
         uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_next >> 3)) : 0u;
         int g_cur = -1;
@@ -189,7 +193,7 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         for (int kb = 0; kb < num_kb && ok; ++kb) {
             const int s = kb % C::kStages;
             const int a = kb % C::kABufs;
-            const int k = kb * kGemmKB + kq * 16;
+            const int k = (kb0 + kb) * kGemmKB + kq * 16;
             const bool live = row_ok && k < K;
             if (live && g_next != g_cur) {
                 g_cur = g_next;
@@ -244,7 +248,12 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int m = m0 + c + j;
-                            if (m < M) Y[(size_t)m * N + nn] = f2h_rn(__uint_as_float(r[j]));
+                            if (m < M) {
+                                if (part)
+                                    part[((size_t)blockIdx.z * M + m) * N + nn] = __uint_as_float(r[j]);
+                                else
+                                    Y[(size_t)m * N + nn] = f2h_rn(__uint_as_float(r[j]));
+                            }
                         }
                     }
                 }
@@ -256,6 +265,240 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Wide form for prefill (M > 128): 256 output channels x 256 tokens per CTA, two
+// dequantised 128-channel A tiles per 64-channel k-block, two 256-column TMEM
+// accumulators.  Every X tile then feeds twice the MMA work of the 128-channel form, and
+// the packed weights have a ring of their own, freed by the dequantisers, so that the X
+// ring (freed by the MMAs) is the only round trip on the MMA's critical path.
+//   warp 0     TMA: X tiles [256 tokens x 64] into the X ring
+//   warp 1     TMEM allocation; one lane issues 8 tcgen05.mma per k-block
+//   warp 2     TMA: packed tiles [256 rows x 8 words] into the W ring
+//   warps 3-18 dequantise (thread = row, 32 codes), then the epilogue
+// ---------------------------------------------------------------------------
+constexpr int kWideRows = 256;
+constexpr int kWideBN = 256;
+constexpr int kWideThreads = 96 + kDequantWarps * 32;
+
+struct GemmWideCfg {
+    static constexpr int kXStages = 4;
+    static constexpr int kWStages = 4;
+    static constexpr int kABufs = 2;
+    static constexpr int kXBytes = kWideBN * 128;              // 256 tokens x 64 fp16
+    static constexpr int kWBytes = kWideRows * 32;             // 256 rows x 8 words
+    static constexpr int kATileBytes = kGemmTileN * 128;       // one 128-channel tile
+    static constexpr int kABytes = 2 * kATileBytes;
+    static constexpr int kXOff = 0;
+    static constexpr int kAOff = kXOff + kXStages * kXBytes;
+    static constexpr int kWOff = kAOff + kABufs * kABytes;
+    static constexpr int kBarOff = kWOff + kWStages * kWBytes;
+    static constexpr int kNumBars = 2 * kXStages + 2 * kWStages + 2 * kABufs + 1;
+    static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kTmemPtrOff + 16 + 1024;
+};
+
+__global__ void __launch_bounds__(kWideThreads, 1)
+gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
+                       const uint16_t* __restrict__ scales, const uint32_t* __restrict__ qzeros, int M, int N, int K,
+                       int G, int zero_point, uint16_t* __restrict__ Y) {
+    using C = GemmWideCfg;
+    using namespace sm100;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    uint64_t* xfull = bars;                         // [kXStages] X landed
+    uint64_t* xempty = xfull + C::kXStages;         // [kXStages] MMA done with the X slot
+    uint64_t* wfull = xempty + C::kXStages;         // [kWStages] packed tile landed
+    uint64_t* wempty = wfull + C::kWStages;         // [kWStages] dequantisers done with it
+    uint64_t* afull = wempty + C::kWStages;         // [kABufs]  dequantised tiles written
+    uint64_t* aempty = afull + C::kABufs;           // [kABufs]  MMA done with them
+    uint64_t* tfull = aempty + C::kABufs;           // accumulators complete
+    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::kTmemPtrOff);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * kWideBN;
+    const int n0 = blockIdx.y * kWideRows;
+    const int num_kb = ceil_div(K, kGemmKB);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kXStages; ++s) {
+            mbar_init(&xfull[s], 1);
+            mbar_init(&xempty[s], 1);
+        }
+        for (int s = 0; s < C::kWStages; ++s) {
+            mbar_init(&wfull[s], 1);
+            mbar_init(&wempty[s], kDequantWarps);
+        }
+        for (int a = 0; a < C::kABufs; ++a) {
+            mbar_init(&afull[a], kDequantWarps);
+            mbar_init(&aempty[a], 1);
+        }
+        mbar_init(tfull, 1);
+        mbar_fence_init();
+        prefetch_tensormap(&tmap_x);
+        prefetch_tensormap(&tmap_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_ptr, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+
+    if (warp == 0 || warp == 2) {
+        if (lane == 0) {
+            // ---------------- TMA: X ring (warp 0) or packed-weight ring (warp 2) ----------------
+            const bool xs = warp == 0;
+            const int S = xs ? C::kXStages : C::kWStages;
+            uint64_t* full = xs ? xfull : wfull;
+            uint64_t* empty = xs ? xempty : wempty;
+            const uint32_t bytes = xs ? C::kXBytes : C::kWBytes;
+            uint8_t* base = smem + (xs ? C::kXOff : C::kWOff);
+            int issued = 0;
+            bool ok = true;
+            for (int kb = 0; kb < num_kb && ok; ++kb) {
+                const int s = kb % S;
+                if (kb >= S) ok = mbar_wait(&empty[s], ((kb / S) - 1) & 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&full[s], bytes);
+                if (xs)
+                    tma_load_2d(base + s * bytes, &tmap_x, &full[s], kb * kGemmKB, m0);
+                else
+                    tma_load_2d(base + s * bytes, &tmap_q, &full[s], kb * (kGemmKB / 8), n0);
+                ++issued;
+            }
+            for (int kb = issued - 1; kb >= 0 && kb >= issued - S; --kb) mbar_wait(&full[kb % S], (kb / S) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            constexpr uint32_t idesc = idesc_f16_f32(kGemmTileN, kWideBN);
+            bool ok = true;
+            for (int kb = 0; kb < num_kb && ok; ++kb) {
+                const int s = kb % C::kXStages;
+                const int a = kb % C::kABufs;
+                ok = mbar_wait(&xfull[s], (kb / C::kXStages) & 1) && mbar_wait(&afull[a], (kb / C::kABufs) & 1);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t abase = smem_u32(smem + C::kAOff + a * C::kABytes);
+                const uint64_t a0 = desc_sw128_kmajor(abase), a1 = desc_sw128_kmajor(abase + C::kATileBytes);
+                const uint64_t bdesc = desc_sw128_kmajor(smem_u32(smem + C::kXOff + s * C::kXBytes));
+#pragma unroll
+                for (int kk = 0; kk < kGemmKB / 16; ++kk) {
+                    mma_f16(tmem, a0 + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+                    mma_f16(tmem + kWideBN, a1 + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+                }
+                mma_commit(&xempty[s]);
+                mma_commit(&aempty[a]);
+            }
+            mma_commit(tfull);   // also on the error path, so that the MMAs drain before TMEM is freed
+            if (!ok) mbar_wait(tfull, 0);
+        }
+    } else {
+        // ---------------- dequantise (thread = channel row, 32 codes), then epilogue ----------------
+        const int d = threadIdx.x - 96;           // 0..511
+        const int row = d & (kWideRows - 1);      // 0..255
+        const int kh = d >> 8;                    // which 32 channels of the k-block
+        const int rt = row >> 7, r = row & 127;
+        const int n = n0 + row;
+        const int ng = K / G;
+        const int nzw = ceil_div(ng, 8);
+        const bool zp = zero_point != 0;
+        const bool row_ok = n < N;
+        const uint16_t* srow = scales + (size_t)(row_ok ? n : 0) * ng;
+        const uint32_t* zrow = qzeros + (size_t)(row_ok ? n : 0) * nzw;
+        int g_next = (kh * 32) / G;
+        uint32_t sc_next = row_ok ? __ldg(srow + g_next) : 0u;
+        uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_next >> 3)) : 0u;
+        int g_cur = -1;
+        uint32_t s2 = 0, zmagic = 0x64006400u, zneg16 = 0;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb && ok; ++kb) {
+            const int s = kb % C::kWStages;
+            const int a = kb % C::kABufs;
+            const int k = kb * kGemmKB + kh * 32;
+            const bool live = row_ok && k < K;
+            if (live && g_next != g_cur) {
+                g_cur = g_next;
+                const uint32_t sc = sc_next;
+                const uint32_t z = zp ? ((zw_next >> (4 * (g_cur & 7))) & 15u) : 8u;
+                s2 = sc | (sc << 16);
+                const uint32_t zm = 0x6400u | z;
+                zmagic = zm | (zm << 16);
+                const uint32_t zn = 0xD000u | (z << 4) | 0x0400u;
+                zneg16 = zn | (zn << 16);
+                const float qz_max = zp ? fmaxf((float)z, 15.0f - (float)z) : 8.0f;
+                if (!(h2f((uint16_t)sc) * qz_max < 65520.0f) && !isnan(h2f((uint16_t)sc))) raise_error(kErrRange);
+            }
+            {   // prefetch the next k-block's group parameters if the group changes
+                const int kn = k + kGemmKB;
+                const int gn = kn / G;
+                if (row_ok && kn < K && gn != g_cur) {
+                    g_next = gn;
+                    sc_next = __ldg(srow + gn);
+                    if (zp) zw_next = __ldg(zrow + (gn >> 3));
+                }
+            }
+            ok = mbar_wait(&wfull[s], (kb / C::kWStages) & 1);
+            if (ok && kb >= C::kABufs) ok = mbar_wait(&aempty[a], ((kb / C::kABufs) - 1) & 1);
+            if (!ok) break;
+            const uint4 packed = *reinterpret_cast<const uint4*>(smem + C::kWOff + s * C::kWBytes + row * 32 + kh * 16);
+            uint4 v[4];
+            v[0] = live ? dequant_word(packed.x, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+            v[1] = live ? dequant_word(packed.y, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+            v[2] = live ? dequant_word(packed.z, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+            v[3] = live ? dequant_word(packed.w, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&wempty[s]);     // the packed words are in registers
+            uint8_t* atile = smem + C::kAOff + a * C::kABytes + rt * C::kATileBytes;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(atile + sw128_offset(r, kh * 4 + c)) = v[c];
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[a]);
+        }
+        if (ok && mbar_wait(tfull, 0)) {
+            tc_fence_after();
+            const int q = warp & 3;                        // TMEM lane quarter this warp may access
+            const int set = (warp - 3) >> 2;               // 0..3: four warps per lane quarter
+            const int ert = set >> 1;                      // accumulator (row tile) of this set
+            const int t0 = (set & 1) * (kWideBN / 2);      // its 128 token columns
+            const int nn = n0 + ert * kGemmTileN + q * 32 + lane;
+            for (int c = 0; c < kWideBN / 2; c += 16) {
+                uint32_t rv[16];
+                tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ert * kWideBN + t0 + c), rv);
+                tmem_ld_wait();
+                if (nn < N) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int m = m0 + t0 + c + j;
+                        if (m < M) Y[(size_t)m * N + nn] = f2h_rn(__uint_as_float(rv[j]));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// Y = fp16(sum over the splits of the fp32 partial sums), the splits added in order.
+__global__ void gemm_split_reduce_kernel(const float* __restrict__ part, int splits, size_t count,
+                                         uint16_t* __restrict__ Y) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x) {
+        float acc = part[i];
+        for (int z = 1; z < splits; ++z) acc += part[(size_t)z * count + i];
+        Y[i] = f2h_rn(acc);
     }
 }
 
@@ -310,7 +553,8 @@ inline bool make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType
 
 template <int BN>
 awq_status launch_gemm_bn(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
-                          const uint32_t* qzeros, int N, int K, int G, int zp, uint16_t* Y, cudaStream_t st) {
+                          const uint32_t* qzeros, int N, int K, int G, int zp, uint16_t* Y, cudaStream_t st,
+                          int splits = 1, float* part = nullptr) {
     using C = GemmCfg<BN>;
     CUtensorMap tx, tq;
     if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)M, (uint64_t)K, BN, kGemmKB,
@@ -322,20 +566,94 @@ awq_status launch_gemm_bn(const uint16_t* X, int M, const uint32_t* qweight, con
     auto kern = gemm_w4a16_kernel<BN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return AWQ_ERR_CUDA;
-    dim3 grid(ceil_div(M, BN), ceil_div(N, kGemmTileN));
+    const int num_kb = ceil_div(K, kGemmKB);
+    if (splits < 1 || part == nullptr) splits = 1;
+    const int kb_per = ceil_div(num_kb, splits);
+    splits = ceil_div(num_kb, kb_per);
+    dim3 grid(ceil_div(M, BN), ceil_div(N, kGemmTileN), splits);
     if (grid.y > 65535u) return AWQ_ERR_UNSUPPORTED;
-    kern<<<grid, kGemmThreads, C::kSmemBytes, st>>>(tx, tq, scales, qzeros, M, N, K, G, zp, Y);
+    kern<<<grid, kGemmThreads, C::kSmemBytes, st>>>(tx, tq, scales, qzeros, M, N, K, G, zp, Y, kb_per,
+                                                    splits > 1 ? part : nullptr);
+    if (splits > 1) {
+        const size_t count = (size_t)M * N;
+        const unsigned blocks = (unsigned)std::min<size_t>((count + 255) / 256, 4096);
+        gemm_split_reduce_kernel<<<blocks, 256, 0, st>>>(part, splits, count, Y);
+    }
     return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+// K splits of the 128-channel form for a batch whose tiles leave SMs idle: enough splits
+// for about two CTAs per SM, each split at least 4 k-blocks (256 channels).  1 = none.
+inline int gemm_splits(int M, int N, int K, int sms) {
+    const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    const long long tiles = (long long)ceil_div(M, bn) * ceil_div(N, kGemmTileN);
+    const int num_kb = ceil_div(K, kGemmKB);
+    if (tiles >= sms) return 1;
+    int s = (int)((2LL * sms + tiles - 1) / tiles);
+    s = std::min(s, std::max(1, num_kb / 4));
+    return std::max(1, s);
+}
+
+// Workspace of the GEMM: the fp32 partial sums of the split-K form (0 when it is not used).
+inline size_t gemm_workspace_bytes(int M, int N, int K, int sms) {
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    const int s = gemm_splits(M, N, K, sms);
+    return s > 1 ? (size_t)s * M * N * 4 : 0;
+}
+
+inline awq_status launch_gemm_wide(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
+                                   const uint32_t* qzeros, int N, int K, int G, int zp, uint16_t* Y, cudaStream_t st) {
+    using C = GemmWideCfg;
+    CUtensorMap tx, tq;
+    if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)M, (uint64_t)K, kWideBN, kGemmKB,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return AWQ_ERR_CUDA;
+    if (!make_tmap_2d(&tq, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)N, (uint64_t)(K / 8), kWideRows,
+                      kGemmKB / 8, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return AWQ_ERR_CUDA;
+    if (cudaFuncSetAttribute(gemm_w4a16_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+        return AWQ_ERR_CUDA;
+    dim3 grid(ceil_div(M, kWideBN), ceil_div(N, kWideRows));
+    if (grid.y > 65535u) return AWQ_ERR_UNSUPPORTED;
+    gemm_w4a16_wide_kernel<<<grid, kWideThreads, C::kSmemBytes, st>>>(tx, tq, scales, qzeros, M, N, K, G, zp, Y);
+    return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+// The wide form does twice the work per tile and, by the k-block rate of the two forms,
+// about kWideGain times the work per unit time; it is used where that beats the wave
+// count of the 128-channel form (one resident CTA per SM for both).
+constexpr double kWideGain = 1.6;
+
+inline bool use_wide_gemm(int M, int N, int sms) {
+    if (M <= 128) return false;
+    const long long mt = ceil_div(M, kWideBN);
+    const long long narrow = mt * ceil_div(N, kGemmTileN), wide = mt * ceil_div(N, kWideRows);
+    const double t_narrow = (double)((narrow + sms - 1) / sms);
+    const double t_wide = (double)((wide + sms - 1) / sms) * 2.0 / kWideGain;
+    return t_wide < t_narrow;
 }
 
 inline awq_status launch_gemm_w4a16(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
                                     const uint32_t* qzeros, int N, int K, int G, int zp, uint16_t* Y, cudaStream_t st,
-                                    int /*sms*/) {
-    if (M <= 16) return launch_gemm_bn<16>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
-    if (M <= 32) return launch_gemm_bn<32>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
-    if (M <= 64) return launch_gemm_bn<64>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
-    if (M <= 128) return launch_gemm_bn<128>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
-    return launch_gemm_bn<256>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
+                                    int sms, void* ws, size_t ws_bytes) {
+    if (use_wide_gemm(M, N, sms)) return launch_gemm_wide(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
+    // split K over the caller's workspace when the tiles alone leave SMs idle (as many
+    // splits as the workspace holds, up to the chosen number)
+    int splits = gemm_splits(M, N, K, sms);
+    if (splits > 1) {
+        const size_t per = (size_t)M * N * 4;
+        const size_t fit = (ws && per) ? ws_bytes / per : 0;
+        splits = (int)std::min<size_t>((size_t)splits, fit);
+    }
+    float* part = splits > 1 ? static_cast<float*>(ws) : nullptr;
+#define AWQ_GEMM_BN(BB) return launch_gemm_bn<BB>(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st, splits, part)
+    if (M <= 16) AWQ_GEMM_BN(16);
+    if (M <= 32) AWQ_GEMM_BN(32);
+    if (M <= 64) AWQ_GEMM_BN(64);
+    if (M <= 128) AWQ_GEMM_BN(128);
+    AWQ_GEMM_BN(256);
+#undef AWQ_GEMM_BN
 }
 
 }  // namespace awq

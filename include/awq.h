@@ -204,7 +204,11 @@ awq_status awq_linear_gemv(const uint16_t* X, int32_t M, const uint32_t* qweight
  * WQLinear_GEMM, the default for batch > 1).  Same result definition as
  * awq_linear_gemv; the weight tile is dequantised to fp16 ((q-zero)*scale16,
  * one rounding) in shared memory and multiplied on the tcgen05 tensor cores with
- * fp32 accumulation in tensor memory.  Any M >= 1.  Needs no workspace.
+ * fp32 accumulation in tensor memory.  Any M >= 1.
+ * Workspace: when the batch gives fewer 128-channel tiles than the GPU has SMs, the
+ * kernel splits K into up to awq_workspace_bytes(AWQ_OP_GEMM, ...) / (4 M N) parts whose
+ * fp32 partial sums go to ws and are added in a fixed order into Y (one fp16 rounding);
+ * ws may be NULL (or small), which only disables the split.
  * Range: each dequantised weight is rounded once to fp16, so it must be finite there:
  * max|q - zero| * scale16 < 65520 for every group (max|q - zero| is max(zero, 15 - zero),
  * or 8 without zero point).  awq_quantize_pack gives that whenever the group's scaled

@@ -101,7 +101,10 @@ def test_scale_search_argument_errors(lib):
 def test_workspace_sizes(lib):
     assert lib.awq_workspace_bytes(0, 1, 4096, 4096, _cfg()) == 0
     assert lib.awq_workspace_bytes(2, 1, 4096, 4096, _cfg()) == 0
-    assert lib.awq_workspace_bytes(3, 512, 4096, 4096, _cfg()) == 0
+    # the GEMM needs a workspace only to split K when its tiles leave SMs idle
+    assert lib.awq_workspace_bytes(3, 2048, 8192, 8192, _cfg()) == 0
+    small = lib.awq_workspace_bytes(3, 16, 4096, 4096, _cfg())
+    assert small > 0 and small % (16 * 4096 * 4) == 0
     a = lib.awq_workspace_bytes(1, 512, 4096, 4096, _cfg())
     b = lib.awq_workspace_bytes(1, 512, 8192, 4096, _cfg())
     assert b > a > 0
