@@ -130,8 +130,14 @@ awq_status awq_quantize_pack(const uint16_t* W, const uint16_t* s, int32_t N, in
     if (!aligned16(W) || !aligned16(qweight) || (s && !aligned16(s))) return AWQ_ERR_INVALID_ARG;
     const long long blocks = (long long)ceil_div(N, kQuantRows) * ceil_div(K, kQuantChunk);
     if (blocks > 0x7fffffffLL) return AWQ_ERR_UNSUPPORTED;
-    quantize_pack_kernel<<<(unsigned)blocks, kQuantThreads, 0, (cudaStream_t)stream>>>(
-        W, s, N, K, cfg.q_group_size, cfg.zero_point, qweight, scales, cfg.zero_point ? qzeros : nullptr);
+    uint32_t* qz = cfg.zero_point ? qzeros : nullptr;
+    const cudaStream_t st_ = (cudaStream_t)stream;
+    switch (cfg.q_group_size) {
+        case 32: quantize_pack_kernel<32><<<(unsigned)blocks, kQuantThreads, 0, st_>>>(W, s, N, K, cfg.zero_point, qweight, scales, qz); break;
+        case 64: quantize_pack_kernel<64><<<(unsigned)blocks, kQuantThreads, 0, st_>>>(W, s, N, K, cfg.zero_point, qweight, scales, qz); break;
+        case 128: quantize_pack_kernel<128><<<(unsigned)blocks, kQuantThreads, 0, st_>>>(W, s, N, K, cfg.zero_point, qweight, scales, qz); break;
+        default: quantize_pack_kernel<256><<<(unsigned)blocks, kQuantThreads, 0, st_>>>(W, s, N, K, cfg.zero_point, qweight, scales, qz); break;
+    }
     stream_order_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
     return launch_status();
 }

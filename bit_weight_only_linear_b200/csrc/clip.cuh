@@ -324,7 +324,7 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
                         for (int e = 0; e < 4; ++e) {
                             const int i = 4 * i4 + e;
                             const float wc = fminf(fmaxf(wsv(i, s4[e]), -cl), cl);     // clipped
-                            rr[i] = rintf(__fmul_rn(wc, p.rc));
+                            rr[i] = rint_magic(__fmul_rn(wc, p.rc));
                             const float dd = __fmaf_rn(rr[i], p.sc, -wc);
                             good = good && (__fmaf_rn(fabsf(wc), 0x1p-22f, fabsf(dd)) < half_sc);
                         }

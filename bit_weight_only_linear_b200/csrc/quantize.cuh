@@ -16,6 +16,26 @@ constexpr int kQuantThreads = 256;                 // 8 elements per thread
 constexpr int kQuantChunk = kQuantThreads * 8;     // 2048 input channels per block
 constexpr float kScaleFloor = 1e-5f;
 
+// The two fp32 products of the fp16 pairs in w and s (each exact: 11-bit x 11-bit
+// significands fit in fp32), by the mixed-precision FMA with a -0 addend: no conversion
+// instructions, and a zero keeps its sign like the plain fp32 product.
+__device__ __forceinline__ void mul_f16x2_f32(uint32_t w, uint32_t s, float& lo, float& hi) {
+    asm("{\n\t.reg .f16 wl, wh, sl, sh;\n\t"
+        "mov.b32 {wl, wh}, %2;\n\t"
+        "mov.b32 {sl, sh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, wl, sl, 0f80000000;\n\t"
+        "fma.rn.f32.f16 %1, wh, sh, 0f80000000;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(w), "r"(s));
+}
+
+// Round to the nearest integer, ties to even, for |x| < 2^22, by adding and removing
+// 1.5 * 2^23 (two FP32 adds instead of a rounding instruction).  Larger |x| gives some
+// value of magnitude >= 2^21, which callers either clamp or re-check.
+__device__ __forceinline__ float rint_magic(float x) {
+    return __fsub_rn(__fadd_rn(x, 12582912.0f), 12582912.0f);
+}
+
 struct GroupParams {
     float sc;     // fp32 value of the fp16 scale
     float rc;     // fl(1 / sc), correctly rounded
@@ -81,15 +101,59 @@ __device__ __forceinline__ void seg_minmax(float& mx, float& mn, int seg) {
 // through shared memory.
 constexpr int kQuantRows = 4;
 
-__global__ void __launch_bounds__(kQuantThreads)
+// Codes of 8 scaled weights with the group's parameters, packed into one word.  The
+// candidate r = rint(ws * rc) is checked against the exact residual r * sc - ws (exact
+// while below sc/2): when |r sc - ws| + |ws| 2^-22 < sc/2, rint(fl(ws / sc)) = r for sure
+// (fl(ws / sc) is within |ws / sc| 2^-24 of ws / sc); otherwise the IEEE division decides.
+// Codes are packed through the fp32 significand: 2^23 + q 16^i has q << 4i in its low
+// bits (exact while q 16^i < 2^23, i.e. codes 0..4 of the word; 5..7 take a second word).
+__device__ __forceinline__ uint32_t pack_codes8(const float (&ws)[8], float sc, float rc, float lo, float hi,
+                                                float off) {
+    float r[8];
+    bool good = true;
+    const float half_sc = 0.5f * sc;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        r[i] = rint_magic(__fmul_rn(ws[i], rc));
+        const float d = __fmaf_rn(r[i], sc, -ws[i]);
+        good = good && (__fmaf_rn(fabsf(ws[i]), 0x1p-22f, fabsf(d)) < half_sc);
+    }
+    if (!good) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r[i] = rintf(__fdiv_rn(ws[i], sc));
+    }
+    uint32_t a = 0, b = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float q = __fadd_rn(fminf(fmaxf(r[i], lo), hi), off);                    // code 0..15
+        const float sh = (float)(1u << (4 * (i < 5 ? i : i - 5)));
+        const uint32_t u = __float_as_uint(__fmaf_rn(q, sh, 8388608.0f));
+        if (i < 5) a |= u; else b |= u;
+    }
+    return (a & 0xFFFFFu) | ((b & 0xFFFu) << 20);
+}
+
+// One block per (4 rows, 2048-channel chunk); thread t owns channels [8t, 8t+8) of the
+// chunk in each of the 4 rows and writes one qweight word per row.  The 4 rows are loaded
+// together; a group's min/max is a shuffle butterfly over its G/8 lanes.  The scale and
+// zero point of each (row, group) are then computed once per warp: a warp holds
+// 4 x 256/G <= 32 such pairs, lane p computes pair p and the lanes fetch their groups'
+// parameters back by shuffles.  The chunk holds whole zero words (2048/G groups, a
+// multiple of 8), packed through shared memory.
+// G is a template parameter: every group index, lane count and shuffle loop is then a
+// compile-time shift or an unrolled sequence (with a run-time G they were integer
+// divisions and loops, a large share of the instructions per element).
+template <int G>
+__global__ void __launch_bounds__(kQuantThreads, 4)
 quantize_pack_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict__ s, int N, int K,
-                     int G, int zero_point, uint32_t* __restrict__ qweight,
+                     int zero_point, uint32_t* __restrict__ qweight,
                      uint16_t* __restrict__ scales, uint32_t* __restrict__ qzeros) {
     __shared__ uint8_t zbuf[kQuantRows][kQuantChunk / 32];
     const int nchunks = ceil_div(K, kQuantChunk);
     const int row0 = (blockIdx.x / nchunks) * kQuantRows;
     const int chunk = blockIdx.x % nchunks;
     const int k0 = chunk * kQuantChunk + threadIdx.x * 8;
+    const int lane = threadIdx.x & 31;
     const bool active = k0 < K;
     const bool zp = zero_point != 0;
     const int ng = K / G;
@@ -100,40 +164,66 @@ quantize_pack_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict_
         wv[r] = make_uint4(0u, 0u, 0u, 0u);
         if (active && row0 + r < N) wv[r] = *reinterpret_cast<const uint4*>(W + (size_t)(row0 + r) * K + k0);
     }
-    float sf[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) sf[i] = 1.0f;
-    if (s != nullptr && active) {
-        const uint4 sv = *reinterpret_cast<const uint4*>(s + k0);
-        const uint16_t* sh = reinterpret_cast<const uint16_t*>(&sv);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sf[i] = h2f(sh[i]);
-    }
-
+    uint4 sv = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);   // s = 1
+    if (s != nullptr && active) sv = *reinterpret_cast<const uint4*>(s + k0);
+    // ws = W s (exact), recomputed from the raw words where needed
+    auto scaled = [&](int r, float (&ws)[8]) {
+        mul_f16x2_f32(wv[r].x, sv.x, ws[0], ws[1]);
+        mul_f16x2_f32(wv[r].y, sv.y, ws[2], ws[3]);
+        mul_f16x2_f32(wv[r].z, sv.z, ws[4], ws[5]);
+        mul_f16x2_f32(wv[r].w, sv.w, ws[6], ws[7]);
+    };
+    // the group extremes of each row
+    float gmx[kQuantRows], gmn[kQuantRows];
 #pragma unroll
     for (int r = 0; r < kQuantRows; ++r) {
-        const int row = row0 + r;                       // uniform over the block
-        const uint16_t* wh = reinterpret_cast<const uint16_t*>(&wv[r]);
         float ws[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ws[i] = s != nullptr ? __fmul_rn(h2f(wh[i]), sf[i]) : h2f(wh[i]);   // exact
+        scaled(r, ws);
         float mx = ws[0], mn = ws[0];
 #pragma unroll
         for (int i = 1; i < 8; ++i) {
             mx = fmaxf(mx, ws[i]);
             mn = fminf(mn, ws[i]);
         }
-        seg_minmax(mx, mn, G >> 3);
-        const GroupParams p = group_params(mx, mn, zp);
-        if (active && row < N) {
-            uint32_t word = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) word |= quant_code(ws[i], p, zp) << (4 * i);
-            qweight[(size_t)row * (K >> 3) + (k0 >> 3)] = word;
+        for (int off = (G >> 3) >> 1; off > 0; off >>= 1) {
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        }
+        gmx[r] = mx;
+        gmn[r] = mn;
+    }
+    // the parameters of pair p = (row p / gpw, group p % gpw of the warp), once per pair
+    constexpr int L = G >> 3;             // lanes per group
+    constexpr int gpw = 32 / L;           // groups per warp and row
+    const int pr = lane / gpw, pg = lane - pr * gpw;
+    float pmx = 0.0f, pmn = 0.0f;
+#pragma unroll
+    for (int r = 0; r < kQuantRows; ++r) {
+        const float a = __shfl_sync(0xffffffffu, gmx[r], pg * L);
+        const float b = __shfl_sync(0xffffffffu, gmn[r], pg * L);
+        if (pr == r) pmx = a, pmn = b;
+    }
+    const GroupParams P = group_params(pmx, pmn, zp);
+    const float plo = zp ? -P.zero : -8.0f, phi = zp ? 15.0f - P.zero : 7.0f;
+    const uint32_t psz = (uint32_t)P.sc16 | ((uint32_t)P.zero << 16);
+#pragma unroll
+    for (int r = 0; r < kQuantRows; ++r) {
+        const int src = r * gpw + lane / L;
+        const float sc = __shfl_sync(0xffffffffu, P.sc, src);
+        const float rc = __shfl_sync(0xffffffffu, P.rc, src);
+        const float lo = __shfl_sync(0xffffffffu, plo, src);
+        const float hi = __shfl_sync(0xffffffffu, phi, src);
+        const uint32_t sz = __shfl_sync(0xffffffffu, psz, src);
+        const int row = row0 + r;                       // uniform over the block
+        if (active && row < N) {
+            float ws[8];
+            scaled(r, ws);
+            qweight[(size_t)row * (K >> 3) + (k0 >> 3)] = pack_codes8(ws, sc, rc, lo, hi, zp ? (float)(sz >> 16) : 8.0f);
             if ((k0 % G) == 0) {
                 const int g = k0 / G;
-                scales[(size_t)row * ng + g] = p.sc16;
-                zbuf[r][(threadIdx.x * 8) / G] = (uint8_t)p.zero;
+                scales[(size_t)row * ng + g] = (uint16_t)(sz & 0xFFFFu);
+                zbuf[r][(threadIdx.x * 8) / G] = (uint8_t)(sz >> 16);
             }
         }
     }

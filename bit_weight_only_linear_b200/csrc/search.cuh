@@ -218,7 +218,7 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 template <int G>
 __global__ void __launch_bounds__(kSearchThreads, 1)
 search_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ W, int M, int N, int K,
-                    int zero_point, const float* __restrict__ s32, const float* __restrict__ rse,
+                    int zero_point, const uint16_t* __restrict__ s_all, const float* __restrict__ rse,
                     const int32_t* __restrict__ eexp, int a0, double* __restrict__ partial) {
     using C = FusedSearchCfg;
     using namespace sm100;
@@ -320,7 +320,7 @@ search_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* 
         const bool row_ok = n < N;
         const bool zp = zero_point != 0;
         const uint16_t* wrow = W + (size_t)(row_ok ? n : 0) * K;
-        const float* sa = s32 + (size_t)y * K;
+        const uint16_t* sa = s_all + (size_t)(a0 + y) * K;     // s of this alpha, fp16
         const float* ra = rse + (size_t)y * K;
         bool ok = true;
         int produced = 0;
@@ -340,18 +340,15 @@ search_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* 
                 wpk[j][0] = v0.x, wpk[j][1] = v0.y, wpk[j][2] = v0.z, wpk[j][3] = v0.w;
                 wpk[j][4] = v1.x, wpk[j][5] = v1.y, wpk[j][6] = v1.z, wpk[j][7] = v1.w;
                 if (k0 < K) {
+                    const uint4 s0 = __ldg(reinterpret_cast<const uint4*>(sa + k0));
+                    const uint4 s1 = __ldg(reinterpret_cast<const uint4*>(sa + k0 + 8));
+                    const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-                    for (int i4 = 0; i4 < 4; ++i4) {
-                        const float4 sv = __ldg(reinterpret_cast<const float4*>(sa + k0) + i4);
-                        const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = i4 * 4 + e;
-                            const uint32_t word = wpk[j][i >> 1];
-                            const float ws = __fmul_rn(h2f((uint16_t)((i & 1) ? (word >> 16) : (word & 0xFFFFu))), s4[e]);
-                            mx = fmaxf(mx, ws);
-                            mn = fminf(mn, ws);
-                        }
+                    for (int h = 0; h < 8; ++h) {
+                        float a, b;
+                        mul_f16x2_f32(wpk[j][h], sw[h], a, b);                  // W s, exact
+                        mx = fmaxf(mx, fmaxf(a, b));
+                        mn = fminf(mn, fminf(a, b));
                     }
                 } else {
                     mx = fmaxf(mx, 0.0f);
@@ -381,21 +378,18 @@ search_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* 
                 if (k0 < K) {
                     float ws[16], rr[16];
                     bool good = true;
+                    const uint4 s0 = __ldg(reinterpret_cast<const uint4*>(sa + k0));
+                    const uint4 s1 = __ldg(reinterpret_cast<const uint4*>(sa + k0 + 8));
+                    const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-                    for (int i4 = 0; i4 < 4; ++i4) {
-                        const float4 sv = __ldg(reinterpret_cast<const float4*>(sa + k0) + i4);
-                        const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
+                    for (int h = 0; h < 8; ++h) mul_f16x2_f32(wpk[j][h], sw[h], ws[2 * h], ws[2 * h + 1]);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = i4 * 4 + e;
-                            const uint32_t word = wpk[j][i >> 1];
-                            ws[i] = __fmul_rn(h2f((uint16_t)((i & 1) ? (word >> 16) : (word & 0xFFFFu))), s4[e]);
-                            // candidate code offset r = rint(ws rc); the residual r sc - ws is exact
-                            // while below sc/2, and then rint(fl(ws / sc)) = r is certain
-                            rr[i] = rintf(__fmul_rn(ws[i], p.rc));
-                            const float dd = __fmaf_rn(rr[i], p.sc, -ws[i]);
-                            good = good && (__fmaf_rn(fabsf(ws[i]), 0x1p-22f, fabsf(dd)) < half_sc);
-                        }
+                    for (int i = 0; i < 16; ++i) {
+                        // candidate code offset r = rint(ws rc); the residual r sc - ws is exact
+                        // while below sc/2, and then rint(fl(ws / sc)) = r is certain
+                        rr[i] = rint_magic(__fmul_rn(ws[i], p.rc));
+                        const float dd = __fmaf_rn(rr[i], p.sc, -ws[i]);
+                        good = good && (__fmaf_rn(fabsf(ws[i]), 0x1p-22f, fabsf(dd)) < half_sc);
                     }
                     if (!good) {
 #pragma unroll
@@ -551,11 +545,11 @@ inline awq_status launch_search_fused(const CUtensorMap& tx, const uint16_t* W, 
     lc.blockDim = dim3(kSearchThreads);
     lc.dynamicSmemBytes = FusedSearchCfg::kSmemBytes;
     lc.stream = st;
-    const float* s32 = w.s32;
+    const uint16_t* s_all = w.s_all;
     const float* rse = w.rse;
     const int32_t* eexp = w.eexp;
     double* partial = w.partial;
-    void* args[] = {const_cast<CUtensorMap*>(&tx), &W, &M, &N, &K, &zp, &s32, &rse, &eexp, &a0, &partial};
+    void* args[] = {const_cast<CUtensorMap*>(&tx), &W, &M, &N, &K, &zp, &s_all, &rse, &eexp, &a0, &partial};
     return cudaLaunchKernelExC(&lc, fn, args) == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
