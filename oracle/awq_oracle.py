@@ -30,9 +30,12 @@ the design notes):
   R5  zero = clamp(rint(-min/scale16), 0, 15) with rint = round-half-even.
   R6  zero_point off: scale = max|ws|/7, q = clamp(rint(ws/scale16), -8, 7) + 8,
       implicit zero 8, no zeros buffer.
-  R7  packing: qweight [N][K/8] uint32, code of (n, k) in bits 4*(k%8).. of
-      word k/8 (little-endian nibbles); zeros [N][ceil(ng/8)] uint32, same
-      nibble order, unused nibbles 0; scales [N][ng] fp16.
+  R7  packing: qweight [N][K/8] uint32, the 8 codes k = 8w .. 8w+7 of word w
+      interleaved over its two 16-bit halves: code 8w+j in nibble CODE_NIBBLE[j] =
+      (0, 4, 1, 5, 2, 6, 3, 7)[j] (bits 4*nibble ..), so that codes k, k+1 sit at the
+      same place of the low and high half; zeros [N][ceil(ng/8)] uint32 in plain
+      little-endian nibble order (group 8v+j in nibble j), unused nibbles 0; scales
+      [N][ng] fp16.
   R8  loss = mean over (m, n) of (sum_k X[m,k] * (deq/s - W)[n,k])^2 in fp64;
       argmin with ties to the smallest alpha; the same G / zero_point as the
       final quantisation.
@@ -161,7 +164,8 @@ def quantize_groups(W16: np.ndarray, s16, G: int, zero_point: bool):
 # ----------------------------------------------------------------------------
 
 def pack_nibbles(codes: np.ndarray) -> np.ndarray:
-    """[R][C] codes 0..15 -> [R][ceil(C/8)] uint32, code j of a word in bits 4j..4j+3."""
+    """Plain packing (the zero points, R7): [R][C] values 0..15 -> [R][ceil(C/8)] uint32,
+    value j of a word in bits 4j..4j+3."""
     codes = np.asarray(codes, dtype=np.uint32)
     R, C = codes.shape
     W = (C + 7) // 8
@@ -184,10 +188,40 @@ def unpack_nibbles(words: np.ndarray, C: int) -> np.ndarray:
     return out.reshape(R, W * 8)[:, :C]
 
 
+# Nibble of code j (0..7) within a qweight word: codes k, k+1 share a position in the
+# two 16-bit halves, so one mask of a word yields the adjacent pair (k, k+1).
+CODE_NIBBLE = (0, 4, 1, 5, 2, 6, 3, 7)
+
+
+def pack_codes(codes: np.ndarray) -> np.ndarray:
+    """qweight packing (R7): [R][C] codes 0..15 -> [R][ceil(C/8)] uint32, code j of a word
+    in nibble CODE_NIBBLE[j]."""
+    codes = np.asarray(codes, dtype=np.uint32)
+    R, C = codes.shape
+    W = (C + 7) // 8
+    padded = np.zeros((R, W * 8), dtype=np.uint32)
+    padded[:, :C] = codes
+    p = padded.reshape(R, W, 8)
+    out = np.zeros((R, W), dtype=np.uint32)
+    for j in range(8):
+        out |= p[:, :, j] << np.uint32(4 * CODE_NIBBLE[j])
+    return out
+
+
+def unpack_codes(words: np.ndarray, C: int) -> np.ndarray:
+    """Inverse of pack_codes: [R][W] uint32 -> [R][C] uint8."""
+    words = np.asarray(words, dtype=np.uint32)
+    R, W = words.shape
+    out = np.zeros((R, W, 8), dtype=np.uint8)
+    for j in range(8):
+        out[:, :, j] = (words >> np.uint32(4 * CODE_NIBBLE[j])) & np.uint32(0xF)
+    return out.reshape(R, W * 8)[:, :C]
+
+
 def quantize_pack(W16: np.ndarray, s16, G: int, zero_point: bool):
     """The awq_quantize_pack operation: (qweight, scales, qzeros or None)."""
     codes, scale16, zeros = quantize_groups(W16, s16, G, zero_point)
-    qweight = pack_nibbles(codes)
+    qweight = pack_codes(codes)
     qzeros = pack_nibbles(zeros) if zero_point else None
     return qweight, scale16, qzeros
 
@@ -196,7 +230,7 @@ def dequantize(qweight, scales, qzeros, K: int, G: int, zero_point: bool) -> np.
     """deq[n][k] = (q - zero) * scale16 in fp64 (exact)."""
     N = qweight.shape[0]
     ng = K // G
-    q = unpack_nibbles(qweight, K).astype(np.float64).reshape(N, ng, G)
+    q = unpack_codes(qweight, K).astype(np.float64).reshape(N, ng, G)
     if zero_point:
         z = unpack_nibbles(qzeros, ng).astype(np.float64)
     else:
@@ -352,7 +386,7 @@ def quantize_pack_clipped(W16, s16, G: int, zero_point: bool, clip_index, n_grid
     ratios = clip_ratios(n_grid, int(idx.max()) + 1)[idx]
     g = clip_groups(scaled_weights(W16, s16).reshape(N, ng, G), ratios)
     q, scale16, zero = quantize_scaled_groups(g, zero_point)
-    qweight = pack_nibbles(q.reshape(N, K).astype(np.uint8))
+    qweight = pack_codes(q.reshape(N, K).astype(np.uint8))
     qzeros = pack_nibbles(zero.astype(np.uint8)) if zero_point else None
     return qweight, scale16, qzeros
 

@@ -24,6 +24,8 @@ MUTATIONS = [
     ("sym_offset", "np.clip(np.rint(g / sc[:, :, None]), -8, 7) + 8", "np.clip(np.rint(g / sc[:, :, None]), -8, 7) + 7"),
     ("no_scale_s", "ws = w32 * s32[None, :]", "ws = w32"),
     ("pack_reversed", "out |= p[:, :, j] << np.uint32(4 * j)", "out |= p[:, :, j] << np.uint32(28 - 4 * j)"),
+    ("code_order_plain", "CODE_NIBBLE = (0, 4, 1, 5, 2, 6, 3, 7)", "CODE_NIBBLE = (0, 1, 2, 3, 4, 5, 6, 7)"),
+    ("code_order_swapped", "CODE_NIBBLE = (0, 4, 1, 5, 2, 6, 3, 7)", "CODE_NIBBLE = (4, 0, 5, 1, 6, 2, 7, 3)"),
     ("absmean_no_abs", "X = np.abs(np.asarray(X16", "X = (np.asarray(X16"),
     ("absmean_divide_K", "/ np.float64(X.shape[0])", "/ np.float64(X.shape[1])"),
     ("alpha_endpoint", "np.arange(n_grid, dtype=np.float64) / np.float64(n_grid)",

@@ -273,12 +273,33 @@ def test_pack_bit_positions():
     assert list(ragged[0]) == [0x00000CA3]
 
 
+def test_code_pack_bit_positions():
+    """qweight order: code j of a word in nibble (0, 4, 1, 5, 2, 6, 3, 7)[j]."""
+    codes = np.array([[1, 2, 3, 4, 5, 6, 7, 8, 15, 0, 0, 0, 0, 0, 0, 9]], dtype=np.uint8)
+    words = O.pack_codes(codes)
+    assert words.dtype == np.uint32
+    assert list(words[0]) == [0x86427531, 0x9000000F]
+    assert list(O.pack_codes(np.array([[3, 10, 12]], dtype=np.uint8))[0]) == [0x000A00C3]
+    # the point of the order: one mask of a word gives an adjacent pair (k, k+1) in its halves
+    c = inputs.random_codes((1, 8 * 64), seed=62)
+    w = O.pack_codes(c)[0]
+    for i, word in enumerate(w):
+        word = int(word)
+        k = 8 * i
+        assert (word & 0xF, (word >> 16) & 0xF) == (c[0, k], c[0, k + 1])
+        assert ((word >> 4) & 0xF, (word >> 20) & 0xF) == (c[0, k + 2], c[0, k + 3])
+        assert ((word >> 8) & 0xF, (word >> 24) & 0xF) == (c[0, k + 4], c[0, k + 5])
+        assert ((word >> 12) & 0xF, (word >> 28) & 0xF) == (c[0, k + 6], c[0, k + 7])
+
+
 def test_pack_unpack_identity():
     for C in (8, 16, 24, 128, 4096, 3, 11):
         c = inputs.random_codes((5, C), seed=60 + C)
         assert np.array_equal(O.unpack_nibbles(O.pack_nibbles(c), C), c)
+        assert np.array_equal(O.unpack_codes(O.pack_codes(c), C), c)
     words = np.random.Generator(np.random.PCG64(61)).integers(0, 2 ** 32, size=(4, 16), dtype=np.uint64).astype(np.uint32)
     assert np.array_equal(O.pack_nibbles(O.unpack_nibbles(words, 128)), words)
+    assert np.array_equal(O.pack_codes(O.unpack_codes(words, 128)), words)
 
 
 def test_quantize_pack_shapes():
@@ -302,7 +323,7 @@ def test_linear_against_naive_loop():
     for zp in (True, False):
         q, s, z = O.quantize_pack(W, None, G, zp)
         y = O.linear(X, q, s, z, K, G, zp)
-        codes = O.unpack_nibbles(q, K)
+        codes = O.unpack_codes(q, K)
         zer = O.unpack_nibbles(z, K // G) if zp else np.full((N, K // G), 8)
         for m in range(M):
             for n in range(N):

@@ -223,7 +223,7 @@ def test_gemm_reports_fp16_overflow(lib):
     scales = np.full((N, K // G), 0.01, dtype=np.float16)
     scales[5, 1] = 5000.0
     zeros = np.zeros((N, K // G), dtype=np.uint8)
-    dq = (to_dev(O.pack_nibbles(codes)), to_dev(scales), to_dev(O.pack_nibbles(zeros)))
+    dq = (to_dev(O.pack_codes(codes)), to_dev(scales), to_dev(O.pack_nibbles(zeros)))
     X = (inputs.activations(16, K, seed=313).astype(np.float32) * np.float32(1e-3)).astype(np.float16)
     lib.linear_gemm(to_dev(X), *dq, G, True)
     with pytest.raises(_awq.AWQError) as err:
@@ -233,7 +233,7 @@ def test_gemm_reports_fp16_overflow(lib):
     dq = (dq[0], to_dev(scales), dq[2])
     y = _run(lib, "gemm", X, dq, G, True)
     lib.device_error()
-    assert_linear_close(y, O.linear(X, O.pack_nibbles(codes), scales, O.pack_nibbles(zeros), K, G, True))
+    assert_linear_close(y, O.linear(X, O.pack_codes(codes), scales, O.pack_nibbles(zeros), K, G, True))
 
 
 def test_gemv_directly_after_quantize_pack(lib):
