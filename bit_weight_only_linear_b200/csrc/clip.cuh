@@ -442,7 +442,7 @@ clip_pack_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict__ s,
         if (active && row < N) {
             uint32_t word = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) word |= quant_code(fminf(fmaxf(ws[i], -cl), cl), p, zp) << (4 * i);
+            for (int i = 0; i < 8; ++i) word |= quant_code(fminf(fmaxf(ws[i], -cl), cl), p, zp) << code_shift(i);
             qweight[(size_t)row * (K >> 3) + (k0 >> 3)] = word;
             if ((k0 % G) == 0) {
                 const int g = k0 / G;

@@ -54,15 +54,17 @@ struct GemmCfg {
     static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
 };
 
-// (q - z) * s for the 8 codes of one word, returned as 4 fp16 pairs in k order.
+// (q - z) * s for the 8 codes of one word, returned as 4 fp16 pairs in k order.  The
+// codes k, k+1 of a word sit at the same nibble of its two 16-bit halves, so each mask
+// below leaves one adjacent pair, already in order.
 __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t zmagic, uint32_t zneg16, uint32_t s2) {
     const uint32_t kMagic = 0x64006400u;     // fp16 1024 in both halves
     const uint32_t kSixteenth = 0x2C002C00u; // fp16 1/16 in both halves
-    uint32_t a = (w & 0x000F000Fu) | kMagic;            // 1024 + q0, 1024 + q4
-    uint32_t b = (w & 0x00F000F0u) | kMagic;            // 1024 + 16 q1, 1024 + 16 q5
+    uint32_t a = (w & 0x000F000Fu) | kMagic;            // 1024 + q0, 1024 + q1
+    uint32_t b = (w & 0x00F000F0u) | kMagic;            // 1024 + 16 q2, 1024 + 16 q3
     const uint32_t w8 = w >> 8;
-    uint32_t c = (w8 & 0x000F000Fu) | kMagic;           // q2, q6
-    uint32_t d = (w8 & 0x00F000F0u) | kMagic;           // q3, q7
+    uint32_t c = (w8 & 0x000F000Fu) | kMagic;           // q4, q5
+    uint32_t d = (w8 & 0x00F000F0u) | kMagic;           // 16 q6, 16 q7
     asm("sub.rn.f16x2 %0, %0, %4;\n\t"                  // q - z (exact)
         "fma.rn.f16x2 %1, %1, %5, %6;\n\t"              // (1024 + 16q)/16 - (64 + z) = q - z (exact)
         "sub.rn.f16x2 %2, %2, %4;\n\t"
@@ -73,12 +75,7 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t zmagic, uint3
         "mul.rn.f16x2 %3, %3, %7;"
         : "+r"(a), "+r"(b), "+r"(c), "+r"(d)
         : "r"(zmagic), "r"(kSixteenth), "r"(zneg16), "r"(s2));
-    uint4 o;
-    o.x = __byte_perm(a, b, 0x5410);   // (k0, k1)
-    o.y = __byte_perm(c, d, 0x5410);   // (k2, k3)
-    o.z = __byte_perm(a, b, 0x7632);   // (k4, k5)
-    o.w = __byte_perm(c, d, 0x7632);   // (k6, k7)
-    return o;
+    return make_uint4(a, b, c, d);   // (k0, k1) (k2, k3) (k4, k5) (k6, k7)
 }
 
 template <int BN>

@@ -19,8 +19,14 @@
 //     3/7.  Products with x are exact in the fp32 accumulator.  The "x1" codes and
 //     the "x16" codes go to two accumulators (D1, D16).
 //   * The k order inside an MMA is free as long as A and B agree: lane (g, t) feeds
-//     the k-slots of its quad with codes of its own word, and X is staged in shared
-//     memory permuted the same way, so no shuffles or byte permutes are needed.
+//     the k-slots of its quad with codes of its own word.  The packed order puts codes
+//     k, k+1 at the same nibble of a word's two halves, so each mask leaves an adjacent
+//     pair: the x1 MMA takes codes (0,1) and (4,5) of the word, the x16 MMA (2,3) and
+//     (6,7); one 16-byte load per lane holds x0..x7 of the word, in natural order.
+//   * X is staged with its 16-byte chunks reordered within each k-step to [j][t]: the
+//     4 lanes of a quad then read 64 contiguous bytes, and with a row pitch of 64 mod
+//     128 bytes the two rows of a quarter-warp fill all 32 banks (in natural order the
+//     lanes t and t+2 would hit the same banks when WT = 4).
 //   * The 4 lanes of a quad cover one k-step of 32*WT consecutive codes (WT = 1, 2, 4
 //     words each for G = 32, 64, >= 128), which always lies inside one group, so after
 //     each k-step the group's scale and zero point are applied once in fp32:
@@ -53,7 +59,7 @@ constexpr int kGemvUnitWords = 8;  // code words per row per lane per unit
 __host__ __device__ constexpr int gemv_words_per_thread(int G) { return G >= 128 ? 4 : G / 32; }
 
 struct GemvSmem {
-    // X permuted: [m][kstep][j][t] uint4, row pitch padded by 64 B; then xsum [m][kstep] fp32;
+    // X as [m][kstep][j][t] uint4, row pitch padded by 64 B; then xsum [m][kstep] fp32;
     // then partials [2 slots][8 warps][16 rows][8 m] fp32; then a 64-byte zero row.
     static __host__ __device__ inline size_t x_pitch(int K) { return (size_t)K * 2 + 64; }
     static __host__ __device__ inline size_t xsum_off(int M, int K) { return (size_t)M * x_pitch(K); }
@@ -196,7 +202,7 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
     for (int i = 0; i < kGemvDepth; ++i)
         if (i < U) load_next(buf[i]);
 
-    // 2. wait for the producer of X, then stage it (permuted) and its per-step sums
+    // 2. wait for the producer of X, then stage it (chunks reordered) and its per-step sums
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const size_t pitch = GemvSmem::x_pitch(K);
     float* xsum = reinterpret_cast<float*>(smem + GemvSmem::xsum_off(M, K));
@@ -219,16 +225,10 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
             if (u < M * kw) {
                 const int m = u / kw;
                 const int word = u - m * kw;
-                // x0..x7 -> (x0,x4) (x2,x6) (x1,x5) (x3,x7): the k-slots of the two MMAs of one word
-                uint4 p;
-                p.x = __byte_perm(v[i].x, v[i].z, 0x5410);
-                p.y = __byte_perm(v[i].y, v[i].w, 0x5410);
-                p.z = __byte_perm(v[i].x, v[i].z, 0x7632);
-                p.w = __byte_perm(v[i].y, v[i].w, 0x7632);
                 const int s = word / (4 * WT);
                 const int r = word - s * 4 * WT;
                 const int tt = r / WT, j = r - tt * WT;
-                *reinterpret_cast<uint4*>(smem + m * pitch + ((size_t)(s * WT + j) * 4 + tt) * 16) = p;
+                *reinterpret_cast<uint4*>(smem + m * pitch + ((size_t)(s * WT + j) * 4 + tt) * 16) = v[i];
             }
         }
     }
@@ -256,6 +256,7 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
     // 3. stream the units; D fragment: y[0] = (row g, col 2t), y[1] = (g, 2t+1),
     //    y[2] = (g+8, 2t), y[3] = (g+8, 2t+1)
     // lanes whose B column is past M read the zero row staged after X
+    // lane (g, t) reads x0..x7 of word t*WT + j of each k-step, staged at chunk j*4 + t
     const uint8_t* xrow = (g < M ? smem + g * pitch : smem + GemvSmem::zero_off(M, K, nsteps)) + t * 16;
     const size_t xstep = g < M ? 64 : 0;
     const int m0 = 2 * t, m1 = 2 * t + 1;
@@ -282,14 +283,14 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
                     const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
                     if (j == 0) {
                         mma_16816_first(d1, wa & 0x000F000Fu, wb & 0x000F000Fu, wa8 & 0x000F000Fu,
-                                        wb8 & 0x000F000Fu, b.x, b.y);
+                                        wb8 & 0x000F000Fu, b.x, b.z);
                         mma_16816_first(d16, wa & 0x00F000F0u, wb & 0x00F000F0u, wa8 & 0x00F000F0u,
-                                        wb8 & 0x00F000F0u, b.z, b.w);
+                                        wb8 & 0x00F000F0u, b.y, b.w);
                     } else {
                         mma_16816(d1, wa & 0x000F000Fu, wb & 0x000F000Fu, wa8 & 0x000F000Fu, wb8 & 0x000F000Fu,
-                                  b.x, b.y);
+                                  b.x, b.z);
                         mma_16816(d16, wa & 0x00F000F0u, wb & 0x00F000F0u, wa8 & 0x00F000F0u, wb8 & 0x00F000F0u,
-                                  b.z, b.w);
+                                  b.y, b.w);
                     }
                 }
                 // fold the k-step's group scale and zero point; k-steps past the end get scale 0
@@ -636,13 +637,13 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
         return;
     }
 
-    // ---------------- consumers: stage X (permuted, zero past K) and its per-step sums ----------------
+    // ---------------- consumers: stage X (chunks reordered, zero past K) and its per-step sums ----------------
     const int cw = warp - kTmaFirstConsumer;          // consumer index 0..7
     const int ct = threadIdx.x - kTmaFirstConsumer * 32;
-    // One bulk copy per X row lands the rows unpermuted; each round then reads 256
-    // 16-byte chunks (16 whole k-steps of one row), and after a barrier writes them
-    // back in place in the order the B fragments want, while the lanes of each
-    // k-step add up its codes' activations.
+    // One bulk copy per X row lands the rows in natural order; each round then reads 256
+    // 16-byte chunks (whole k-steps of one row), and after a barrier writes them back in
+    // place in the [j][t] order the B fragments read, while the lanes of each k-step add
+    // up its activations.
     const size_t pitch = GemvSmem::x_pitch(L.Kp);
     uint8_t* xs = smem + L.x();
     float* xsum = reinterpret_cast<float*>(smem + L.xsum());
@@ -664,16 +665,11 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
             const int m = u0 / kwp;
             const int word = u - m * kwp;
             uint4* row = reinterpret_cast<uint4*>(xs + m * pitch);
-            const uint4 v = word < kwv ? row[word] : make_uint4(0u, 0u, 0u, 0u);
+            const uint4 v = word < kwv ? row[word] : make_uint4(0u, 0u, 0u, 0u);   // zero past K
             asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
-            uint4 p;
-            p.x = __byte_perm(v.x, v.z, 0x5410);
-            p.y = __byte_perm(v.y, v.w, 0x5410);
-            p.z = __byte_perm(v.x, v.z, 0x7632);
-            p.w = __byte_perm(v.y, v.w, 0x7632);
             const int s = word / TPS, r = word % TPS;
             const int tt = r / WT, j = r % WT;
-            row[(s * WT + j) * 4 + tt] = p;
+            row[(s * WT + j) * 4 + tt] = v;
             const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
             float acc = 0.0f;
 #pragma unroll
@@ -694,6 +690,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
     constexpr int R = G >= kStepCodes ? G / kStepCodes : 1;   // k-steps per group
     const int g = lane >> 2, t = lane & 3;
     const uint32_t sbase = smem_u32(smem);
+    // lane (g, t) reads x0..x7 of word t*WT + j of each k-step, staged at chunk j*4 + t
     const uint32_t xrow = smem_u32(xs + (g < M ? g : 0) * pitch) + t * 16 + (uint32_t)(cw * Q * WT * 64);
     const int m0 = 2 * t, m1 = 2 * t + 1;
     const uint32_t xs0 = smem_u32(xsum + (m0 < M ? m0 : 0) * nstepsp) + (uint32_t)(cw * Q * 4);
@@ -737,14 +734,14 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
                     const uint32_t a8 = a >> 8, b8 = bb >> 8;
                     if (j == 0) {
                         mma_16816_first(d1[q], a & 0x000F000Fu, bb & 0x000F000Fu, a8 & 0x000F000Fu,
-                                        b8 & 0x000F000Fu, b.x, b.y);
+                                        b8 & 0x000F000Fu, b.x, b.z);
                         mma_16816_first(d16[q], a & 0x00F000F0u, bb & 0x00F000F0u, a8 & 0x00F000F0u,
-                                        b8 & 0x00F000F0u, b.z, b.w);
+                                        b8 & 0x00F000F0u, b.y, b.w);
                     } else {
                         mma_16816(d1[q], a & 0x000F000Fu, bb & 0x000F000Fu, a8 & 0x000F000Fu, b8 & 0x000F000Fu,
-                                  b.x, b.y);
+                                  b.x, b.z);
                         mma_16816(d16[q], a & 0x00F000F0u, bb & 0x00F000F0u, a8 & 0x00F000F0u,
-                                  b8 & 0x00F000F0u, b.z, b.w);
+                                  b8 & 0x00F000F0u, b.y, b.w);
                     }
                 }
             }

@@ -12,6 +12,11 @@
 
 namespace awq {
 
+// Bit position of code j (0..7) in a qweight word: codes k, k+1 share a nibble position
+// in the low and high 16-bit halves (nibbles 0, 4, 1, 5, 2, 6, 3, 7), so one mask of the
+// word yields the adjacent pair (k, k+1) as the tensor-core fragments take it.
+__host__ __device__ constexpr int code_shift(int j) { return 4 * ((j >> 1) + 4 * (j & 1)); }   // 0,16,4,20,8,24,12,28
+
 constexpr int kQuantThreads = 256;                 // 8 elements per thread
 constexpr int kQuantChunk = kQuantThreads * 8;     // 2048 input channels per block
 constexpr float kScaleFloor = 1e-5f;
@@ -105,8 +110,9 @@ constexpr int kQuantRows = 4;
 // candidate r = rint(ws * rc) is checked against the exact residual r * sc - ws (exact
 // while below sc/2): when |r sc - ws| + |ws| 2^-22 < sc/2, rint(fl(ws / sc)) = r for sure
 // (fl(ws / sc) is within |ws / sc| 2^-24 of ws / sc); otherwise the IEEE division decides.
-// Codes are packed through the fp32 significand: 2^23 + q 16^i has q << 4i in its low
-// bits (exact while q 16^i < 2^23, i.e. codes 0..4 of the word; 5..7 take a second word).
+// Codes are packed through the fp32 significand: 2^23 + q 2^b has q << b in its low bits
+// (exact while q 2^b < 2^23, i.e. bit positions up to 16; positions 20, 24, 28 take a
+// second word shifted by 20).
 __device__ __forceinline__ uint32_t pack_codes8(const float (&ws)[8], float sc, float rc, float lo, float hi,
                                                 float off) {
     float r[8];
@@ -126,9 +132,10 @@ __device__ __forceinline__ uint32_t pack_codes8(const float (&ws)[8], float sc, 
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const float q = __fadd_rn(fminf(fmaxf(r[i], lo), hi), off);                    // code 0..15
-        const float sh = (float)(1u << (4 * (i < 5 ? i : i - 5)));
-        const uint32_t u = __float_as_uint(__fmaf_rn(q, sh, 8388608.0f));
-        if (i < 5) a |= u; else b |= u;
+        const int sh = code_shift(i);
+        const float m = (float)(1u << (sh <= 16 ? sh : sh - 20));
+        const uint32_t u = __float_as_uint(__fmaf_rn(q, m, 8388608.0f));
+        if (sh <= 16) a |= u; else b |= u;
     }
     return (a & 0xFFFFFu) | ((b & 0xFFFu) << 20);
 }
