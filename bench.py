@@ -407,6 +407,96 @@ def time_decode_e2e(awq, torch, layers, steps):
     return med(eager), med(graphed), h2d, d2h
 
 
+def time_decode_e2e_pipelined(awq, torch, layers, steps, per_graph=8, depth=2):
+    """The same end-to-end step with its copies overlapped across steps: step i's inputs
+    go host->device on an upload stream while step i-1's GEMVs run, and its outputs come
+    back device->host on a download stream while step i+1's GEMVs run.  Every step still
+    copies its own inputs from pinned memory and reads its own outputs into pinned
+    memory; `depth` device/host buffer pairs carry the steps in flight, and events order
+    each buffer's reuse.  Returns (eager ms, graph ms) for `steps` steps: `eager` issues
+    every call from Python; `graph` replays a captured run of `per_graph` steps (one
+    replay covers every weight rotation twice; the pipeline fills and drains once per
+    replay)."""
+    ks = [L["K"] for L in layers]
+    ns = [L["N"] for L in layers]
+    xo = np.cumsum([0] + ks)
+    yo = np.cumsum([0] + ns)
+    x_np = np.concatenate([L["x_host"].reshape(-1) for L in layers])
+    x_host = [torch.from_numpy(x_np.copy()).pin_memory() for _ in range(depth)]
+    y_host = [torch.empty(sum(ns), dtype=torch.float16).pin_memory() for _ in range(depth)]
+    x_dev = [torch.empty(x_np.size, dtype=torch.float16, device="cuda") for _ in range(depth)]
+    y_dev = [torch.empty(sum(ns), dtype=torch.float16, device="cuda") for _ in range(depth)]
+    xs = [[x[xo[i]:xo[i + 1]].view(1, ks[i]) for i in range(len(layers))] for x in x_dev]
+    ys = [[y[yo[i]:yo[i + 1]].view(1, ns[i]) for i in range(len(layers))] for y in y_dev]
+    comp, up, down = torch.cuda.current_stream(), torch.cuda.Stream(), torch.cuda.Stream()
+
+    def run(n, start):
+        """Issue steps start .. start+n-1 on the three streams (inside a capture too)."""
+        ev = {k: [torch.cuda.Event() for _ in range(depth)] for k in ("up", "comp", "down")}
+        seen = {k: [False] * depth for k in ev}
+        fork = torch.cuda.Event()
+        fork.record(comp)
+        up.wait_event(fork)
+        down.wait_event(fork)
+        for i in range(start, start + n):
+            b, r = i % depth, i % ROTATIONS
+            with torch.cuda.stream(up):
+                if seen["comp"][b]:
+                    up.wait_event(ev["comp"][b])          # the GEMVs that read x_dev[b] are done
+                x_dev[b].copy_(x_host[b], non_blocking=True)
+                ev["up"][b].record(up)
+                seen["up"][b] = True
+            with torch.cuda.stream(comp):
+                comp.wait_event(ev["up"][b])
+                if seen["down"][b]:
+                    comp.wait_event(ev["down"][b])        # y_dev[b] has been read back
+                for L, x, y in zip(layers, xs[b], ys[b]):
+                    q, sc, z = L["copies"][r]
+                    awq.linear_gemv(x, q, sc, z, G, ZP, out=y)
+                ev["comp"][b].record(comp)
+                seen["comp"][b] = True
+            with torch.cuda.stream(down):
+                down.wait_event(ev["comp"][b])
+                y_host[b].copy_(y_dev[b], non_blocking=True)
+                ev["down"][b].record(down)
+                seen["down"][b] = True
+        comp.wait_stream(up)
+        comp.wait_stream(down)
+
+    run(8, 0)
+    torch.cuda.synchronize()
+    eager = []
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(comp)
+        run(steps, 0)
+        e1.record(comp)
+        torch.cuda.synchronize()
+        eager.append(e0.elapsed_time(e1))
+    gstream = torch.cuda.Stream()
+    with torch.cuda.stream(gstream):
+        comp = gstream
+        run(per_graph, 0)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gstream):
+            run(per_graph, 0)
+        g.replay()
+        torch.cuda.synchronize()
+        reps = max(1, -(-steps // per_graph))
+        graphed = []
+        for _ in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(gstream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(gstream)
+            torch.cuda.synchronize()
+            graphed.append(e0.elapsed_time(e1) * steps / (reps * per_graph))
+        del g
+    return med(eager), med(graphed)
+
+
 def measure_single_gemv(awq, torch, peaks):
     """One 4096x4096 GEMV at M=1 (G=128, zero point): 32 rotated weight copies."""
     K = N = 4096
@@ -731,13 +821,22 @@ def run_ours(args):
     eager_ms, graph_ms, h2d, d2h = time_decode_e2e(awq, torch, layers, e2e_steps)
     eager_ms = _max_over_ranks(world, eager_ms)
     graph_ms = _max_over_ranks(world, graph_ms)
-    e2e = {"value": round(aggregate_gbs(world, step_bytes, e2e_steps, eager_ms), 1), "unit": "GB/s",
+    pipe_ms, pipe_graph_ms = time_decode_e2e_pipelined(awq, torch, layers, e2e_steps)
+    pipe_ms = _max_over_ranks(world, pipe_ms)
+    pipe_graph_ms = _max_over_ranks(world, pipe_graph_ms)
+    e2e = {"value": round(aggregate_gbs(world, step_bytes, e2e_steps, pipe_graph_ms), 1), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "how": "per step: one pinned H2D copy of the 4 input vectors, 4 awq_linear_gemv calls from Python "
-                  "through the C ABI, one D2H copy of the 4 outputs; median of 5 trials",
-           "graph_value": round(aggregate_gbs(world, step_bytes, e2e_steps, graph_ms), 1),
-           "graph_how": "the same copies and calls captured once per weight rotation in a CUDA graph, "
-                        "one graph replay per step"}
+           "how": "per step: one pinned H2D copy of the 4 input vectors, 4 awq_linear_gemv calls through the C ABI, "
+                  "one D2H copy of the 4 outputs into pinned memory; the uploads and downloads run on their own "
+                  "streams, overlapped with the GEMVs of the neighbouring steps (2 buffers in flight); the calls "
+                  "of 8 steps captured in one CUDA graph, replayed; median of 5 trials",
+           "pipelined_eager_value": round(aggregate_gbs(world, step_bytes, e2e_steps, pipe_ms), 1),
+           "pipelined_eager_how": "the same pipelined steps, every call issued from Python",
+           "serial_value": round(aggregate_gbs(world, step_bytes, e2e_steps, eager_ms), 1),
+           "serial_how": "copies and calls in order on one stream, every call issued from Python",
+           "serial_graph_value": round(aggregate_gbs(world, step_bytes, e2e_steps, graph_ms), 1),
+           "serial_graph_how": "the serial step captured once per weight rotation in a CUDA graph, "
+                               "one graph replay per step"}
 
     for L in layers:
         L.clear()

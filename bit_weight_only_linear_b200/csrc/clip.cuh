@@ -247,7 +247,10 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
             if (lane == 0) mbar_arrive(&accempty[acc]);
             double* rb = red + (size_t)(t & 1) * kClipRows * 4;
             rb[(q4 * 32 + lane) * 4 + set] = part;
-            asm volatile("bar.sync 1, %0;" ::"n"(kClipProducerWarps * 32) : "memory");
+            // only the four warps of this TMEM lane quarter meet here (named barrier 2 + q4):
+            // the row sums need their four parts, and the buffer of tile t is written again
+            // at tile t + 2 only by warps that have passed this barrier at tile t + 1
+            asm volatile("bar.sync %0, %1;" ::"r"(2 + q4), "n"(4 * 32) : "memory");
             if (set == 0) {
                 const int rr = q4 * 32 + lane;
                 const int nn = n0 + rr;

@@ -27,6 +27,9 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
+// Workspace carving: sizes rounded up to 256 bytes.
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
 // Wait limit for every spin in this library: 2 s of wall time.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

@@ -22,7 +22,9 @@
 //     the k-slots of its quad with codes of its own word.  The packed order puts codes
 //     k, k+1 at the same nibble of a word's two halves, so each mask leaves an adjacent
 //     pair: the x1 MMA takes codes (0,1) and (4,5) of the word, the x16 MMA (2,3) and
-//     (6,7); one 16-byte load per lane holds x0..x7 of the word, in natural order.
+//     (6,7).  One 16-byte load per lane holds x0..x7 of the word, staged as
+//     (x0 x1, x4 x5, x2 x3, x6 x7) so that each MMA's B operand is a register pair
+//     as loaded.
 //   * X is staged with its 16-byte chunks reordered within each k-step to [j][t]: the
 //     4 lanes of a quad then read 64 contiguous bytes, and with a row pitch of 64 mod
 //     128 bytes the two rows of a quarter-warp fill all 32 banks (in natural order the
@@ -228,7 +230,8 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
                 const int s = word / (4 * WT);
                 const int r = word - s * 4 * WT;
                 const int tt = r / WT, j = r - tt * WT;
-                *reinterpret_cast<uint4*>(smem + m * pitch + ((size_t)(s * WT + j) * 4 + tt) * 16) = v[i];
+                *reinterpret_cast<uint4*>(smem + m * pitch + ((size_t)(s * WT + j) * 4 + tt) * 16) =
+                    make_uint4(v[i].x, v[i].z, v[i].y, v[i].w);
             }
         }
     }
@@ -283,14 +286,14 @@ gemv_mma_kernel(const uint16_t* __restrict__ X, int M, const uint32_t* __restric
                     const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
                     if (j == 0) {
                         mma_16816_first(d1, wa & 0x000F000Fu, wb & 0x000F000Fu, wa8 & 0x000F000Fu,
-                                        wb8 & 0x000F000Fu, b.x, b.z);
+                                        wb8 & 0x000F000Fu, b.x, b.y);
                         mma_16816_first(d16, wa & 0x00F000F0u, wb & 0x00F000F0u, wa8 & 0x00F000F0u,
-                                        wb8 & 0x00F000F0u, b.y, b.w);
+                                        wb8 & 0x00F000F0u, b.z, b.w);
                     } else {
                         mma_16816(d1, wa & 0x000F000Fu, wb & 0x000F000Fu, wa8 & 0x000F000Fu, wb8 & 0x000F000Fu,
-                                  b.x, b.z);
+                                  b.x, b.y);
                         mma_16816(d16, wa & 0x00F000F0u, wb & 0x00F000F0u, wa8 & 0x00F000F0u, wb8 & 0x00F000F0u,
-                                  b.y, b.w);
+                                  b.z, b.w);
                     }
                 }
                 // fold the k-step's group scale and zero point; k-steps past the end get scale 0
@@ -669,7 +672,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
             asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
             const int s = word / TPS, r = word % TPS;
             const int tt = r / WT, j = r % WT;
-            row[(s * WT + j) * 4 + tt] = v;
+            row[(s * WT + j) * 4 + tt] = make_uint4(v.x, v.z, v.y, v.w);
             const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
             float acc = 0.0f;
 #pragma unroll
@@ -734,14 +737,14 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint16_t* __re
                     const uint32_t a8 = a >> 8, b8 = bb >> 8;
                     if (j == 0) {
                         mma_16816_first(d1[q], a & 0x000F000Fu, bb & 0x000F000Fu, a8 & 0x000F000Fu,
-                                        b8 & 0x000F000Fu, b.x, b.z);
+                                        b8 & 0x000F000Fu, b.x, b.y);
                         mma_16816_first(d16[q], a & 0x00F000F0u, bb & 0x00F000F0u, a8 & 0x00F000F0u,
-                                        b8 & 0x00F000F0u, b.y, b.w);
+                                        b8 & 0x00F000F0u, b.z, b.w);
                     } else {
                         mma_16816(d1[q], a & 0x000F000Fu, bb & 0x000F000Fu, a8 & 0x000F000Fu, b8 & 0x000F000Fu,
-                                  b.x, b.z);
+                                  b.x, b.y);
                         mma_16816(d16[q], a & 0x00F000F0u, bb & 0x00F000F0u, a8 & 0x00F000F0u,
-                                  b8 & 0x00F000F0u, b.y, b.w);
+                                  b8 & 0x00F000F0u, b.z, b.w);
                     }
                 }
             }

@@ -106,38 +106,50 @@ __device__ __forceinline__ void seg_minmax(float& mx, float& mn, int seg) {
 // through shared memory.
 constexpr int kQuantRows = 4;
 
-// Codes of 8 scaled weights with the group's parameters, packed into one word.  The
-// candidate r = rint(ws * rc) is checked against the exact residual r * sc - ws (exact
-// while below sc/2): when |r sc - ws| + |ws| 2^-22 < sc/2, rint(fl(ws / sc)) = r for sure
-// (fl(ws / sc) is within |ws / sc| 2^-24 of ws / sc); otherwise the IEEE division decides.
-// Codes are packed through the fp32 significand: 2^23 + q 2^b has q << b in its low bits
-// (exact while q 2^b < 2^23, i.e. bit positions up to 16; positions 20, 24, 28 take a
-// second word shifted by 20).
-__device__ __forceinline__ uint32_t pack_codes8(const float (&ws)[8], float sc, float rc, float lo, float hi,
-                                                float off) {
-    float r[8];
+// Codes of 8 scaled weights of one group, packed into one word, from the group's
+// reciprocal scale rc = fl(1/sc) and its clamp bounds in the biased domain below.
+//  * Rounding: t = fl(q + 1.5 * 2^23) with q = fl(ws * rc) holds rint(q) (ties to even)
+//    as an integer in its significand while |q| < 2^22, and r = t - 1.5 * 2^23 and
+//    e = q - r are exact.
+//  * Exactness: q is within |ws/sc| (2^-23 + 2^-48) of ws/sc and fl(ws/sc) within
+//    |ws/sc| 2^-24, so for |ws/sc| <= 33 the two differ by less than 2^-17.  Then
+//    |e| < 1/2 - 2^-17 puts fl(ws/sc) strictly inside r's rounding interval, so
+//    rint(fl(ws/sc)) = r.  When |q| >= 32 the code is clamped to the same end of the
+//    range for any rounding of the quotient, so the test may pass there too.  If any of
+//    the 8 fails, all 8 take the IEEE division.
+//  * Clamp and pack: the clamp to [lo, hi] happens on t, against the bounds
+//    1.5 * 2^23 + lo and 1.5 * 2^23 + hi.  Near 1.5 * 2^23 the bit pattern of a float is
+//    linear in its integer value, so bits(t) - (bits(1.5 * 2^23) - off) is the code,
+//    with off = zero, or 8 when symmetric.  The 8 codes are summed at their nibbles from
+//    the raw bits (mod 2^32), and the 8 copies of that bias are removed at once:
+//    bias * 0x11111111.  The codes lie in 0..15 at distinct nibbles, so no carry crosses
+//    a nibble.
+constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23
+constexpr uint32_t kMagicBits = 0x4B400000u;   // its bit pattern
+
+__device__ __forceinline__ uint32_t pack_codes8(const float (&ws)[8], float rc, uint32_t sz, bool zp) {
+    float t[8];
     bool good = true;
-    const float half_sc = 0.5f * sc;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        r[i] = rint_magic(__fmul_rn(ws[i], rc));
-        const float d = __fmaf_rn(r[i], sc, -ws[i]);
-        good = good && (__fmaf_rn(fabsf(ws[i]), 0x1p-22f, fabsf(d)) < half_sc);
+        const float q = __fmul_rn(ws[i], rc);
+        t[i] = __fadd_rn(q, kMagic);
+        const float e = __fsub_rn(q, __fsub_rn(t[i], kMagic));
+        good = good && (fabsf(e) < 0.5f - 0x1p-17f);
     }
     if (!good) {
+        const float sc = h2f((uint16_t)(sz & 0xFFFFu));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) r[i] = rintf(__fdiv_rn(ws[i], sc));
+        for (int i = 0; i < 8; ++i) t[i] = __fadd_rn(rintf(__fdiv_rn(ws[i], sc)), kMagic);
     }
-    uint32_t a = 0, b = 0;
+    const uint32_t zero = sz >> 16;
+    const uint32_t off = zp ? zero : 8u;
+    const float tlo = __uint_as_float(kMagicBits - off);           // 1.5 * 2^23 + lo
+    const float thi = __uint_as_float(kMagicBits + 15u - off);     // 1.5 * 2^23 + hi
+    uint32_t acc = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float q = __fadd_rn(fminf(fmaxf(r[i], lo), hi), off);                    // code 0..15
-        const int sh = code_shift(i);
-        const float m = (float)(1u << (sh <= 16 ? sh : sh - 20));
-        const uint32_t u = __float_as_uint(__fmaf_rn(q, m, 8388608.0f));
-        if (sh <= 16) a |= u; else b |= u;
-    }
-    return (a & 0xFFFFFu) | ((b & 0xFFFu) << 20);
+    for (int i = 0; i < 8; ++i) acc += __float_as_uint(fminf(fmaxf(t[i], tlo), thi)) << code_shift(i);
+    return acc - (kMagicBits - off) * 0x11111111u;
 }
 
 // One block per (4 rows, 2048-channel chunk); thread t owns channels [8t, 8t+8) of the
@@ -173,24 +185,20 @@ quantize_pack_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict_
     }
     uint4 sv = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);   // s = 1
     if (s != nullptr && active) sv = *reinterpret_cast<const uint4*>(s + k0);
-    // ws = W s (exact), recomputed from the raw words where needed
-    auto scaled = [&](int r, float (&ws)[8]) {
-        mul_f16x2_f32(wv[r].x, sv.x, ws[0], ws[1]);
-        mul_f16x2_f32(wv[r].y, sv.y, ws[2], ws[3]);
-        mul_f16x2_f32(wv[r].z, sv.z, ws[4], ws[5]);
-        mul_f16x2_f32(wv[r].w, sv.w, ws[6], ws[7]);
-    };
-    // the group extremes of each row
+    // ws = W s (exact), kept for both passes; the group extremes of each row
+    float ws[kQuantRows][8];
     float gmx[kQuantRows], gmn[kQuantRows];
 #pragma unroll
     for (int r = 0; r < kQuantRows; ++r) {
-        float ws[8];
-        scaled(r, ws);
-        float mx = ws[0], mn = ws[0];
+        mul_f16x2_f32(wv[r].x, sv.x, ws[r][0], ws[r][1]);
+        mul_f16x2_f32(wv[r].y, sv.y, ws[r][2], ws[r][3]);
+        mul_f16x2_f32(wv[r].z, sv.z, ws[r][4], ws[r][5]);
+        mul_f16x2_f32(wv[r].w, sv.w, ws[r][6], ws[r][7]);
+        float mx = ws[r][0], mn = ws[r][0];
 #pragma unroll
         for (int i = 1; i < 8; ++i) {
-            mx = fmaxf(mx, ws[i]);
-            mn = fminf(mn, ws[i]);
+            mx = fmaxf(mx, ws[r][i]);
+            mn = fminf(mn, ws[r][i]);
         }
 #pragma unroll
         for (int off = (G >> 3) >> 1; off > 0; off >>= 1) {
@@ -212,21 +220,15 @@ quantize_pack_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict_
         if (pr == r) pmx = a, pmn = b;
     }
     const GroupParams P = group_params(pmx, pmn, zp);
-    const float plo = zp ? -P.zero : -8.0f, phi = zp ? 15.0f - P.zero : 7.0f;
     const uint32_t psz = (uint32_t)P.sc16 | ((uint32_t)P.zero << 16);
 #pragma unroll
     for (int r = 0; r < kQuantRows; ++r) {
         const int src = r * gpw + lane / L;
-        const float sc = __shfl_sync(0xffffffffu, P.sc, src);
         const float rc = __shfl_sync(0xffffffffu, P.rc, src);
-        const float lo = __shfl_sync(0xffffffffu, plo, src);
-        const float hi = __shfl_sync(0xffffffffu, phi, src);
         const uint32_t sz = __shfl_sync(0xffffffffu, psz, src);
         const int row = row0 + r;                       // uniform over the block
         if (active && row < N) {
-            float ws[8];
-            scaled(r, ws);
-            qweight[(size_t)row * (K >> 3) + (k0 >> 3)] = pack_codes8(ws, sc, rc, lo, hi, zp ? (float)(sz >> 16) : 8.0f);
+            qweight[(size_t)row * (K >> 3) + (k0 >> 3)] = pack_codes8(ws[r], rc, sz, zp);
             if ((k0 % G) == 0) {
                 const int g = k0 / G;
                 scales[(size_t)row * ng + g] = (uint16_t)(sz & 0xFFFFu);

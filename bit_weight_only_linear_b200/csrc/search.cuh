@@ -61,8 +61,6 @@ struct FusedSearchCfg {
     static constexpr int kSmemBytes = kTmemPtrOff + 16 + 1024;  // + slack to align the base to 1024
 };
 
-inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-
 // Scratch of one search.  `slots` alpha tables (s as fp32, fl(1/s) 2^e) are held at a
 // time: all of them for awq_scale_search, one for the chunked form.
 struct SearchWorkspace {
@@ -325,6 +323,17 @@ search_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* 
         bool ok = true;
         int produced = 0;
         for (int kb0 = 0; kb0 < num_kb && ok; kb0 += U) {
+            // the next unit's lines of W, s and rse into L1 while this unit is computed (its
+            // loads would otherwise wait on L2 at the top of every unit)
+#pragma unroll
+            for (int j = 0; j < U; ++j) {
+                const int k0n = (kb0 + U + j) * 64 + qq * 16;
+                if (k0n < K) {
+                    if (row_ok) prefetch_l1(wrow + k0n);
+                    prefetch_l1(sa + k0n);
+                    prefetch_l1(ra + k0n);
+                }
+            }
             // pass 1: the unit's weights (kept packed) and the group's extremes of W s
             uint32_t wpk[U][8];
             float mx = -INFINITY, mn = INFINITY;
@@ -540,6 +549,10 @@ inline awq_status launch_search_fused(const CUtensorMap& tx, const uint16_t* W, 
                                       const SearchWorkspace& w, int a0, int count, cudaStream_t st) {
     const void* fn = search_fused_fn(G);
     if (!prepare_kernel(fn)) return AWQ_ERR_CUDA;
+    // carve out no more shared memory than the block needs (196 of 228 KB), so that L1
+    // keeps room for the producers' prefetched lines (one unit: up to 33 KB at G = 128)
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 86) != cudaSuccess)
+        return AWQ_ERR_CUDA;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(ceil_div(N, kSearchRows), count, ceil_div(M, kSearchTokChunk));
     lc.blockDim = dim3(kSearchThreads);
