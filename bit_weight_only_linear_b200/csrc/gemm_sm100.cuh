@@ -266,7 +266,7 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
 }
 
 // ---------------------------------------------------------------------------
-// Wide form for prefill (M > 128): 256 output channels x 256 tokens per tile, two
+// Wide form for prefill (M > 128): 256 output channels x 256 tokens per CTA, two
 // dequantised 128-channel A tiles per 64-channel k-block, two 256-column TMEM
 // accumulators.  Every X tile then feeds twice the MMA work of the 128-channel form, and
 // the packed weights have a ring of their own, freed by the dequantisers, so that the X
@@ -275,28 +275,10 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
 //   warp 1     TMEM allocation; one lane issues 8 tcgen05.mma per k-block
 //   warp 2     TMA: packed tiles [256 rows x 8 words] into the W ring
 //   warps 3-18 dequantise (thread = row, 32 codes), then the epilogue
-//
-// Work of a CTA: a range of the flattened (tile, k-block) space, walked as fragments
-// (the part of the range inside one tile).  Data-parallel launch: CTA b takes the whole
-// tile tile0 + b.  Stream-K launch (the tiles of a last, partial wave): the sk_tiles
-// tiles from tile0 on are cut into gridDim.x equal ranges of k-blocks (gridDim.x >=
-// sk_tiles, so a range meets at most two tiles).  A tile is then shared by 2..5 CTAs;
-// each writes its fp32 accumulator to a workspace slot and counts its arrival, and the
-// last to arrive adds the slots of all contributors in k order and writes Y.  Nothing
-// waits for another CTA, so the launch needs no co-residency.
 // ---------------------------------------------------------------------------
 constexpr int kWideRows = 256;
 constexpr int kWideBN = 256;
 constexpr int kWideThreads = 96 + kDequantWarps * 32;
-constexpr int kWidePartFloats = 2 * kWideBN * kGemmTileN;   // [512 TMEM columns][128 lanes] fp32
-
-struct WideSched {
-    int tiles_m;          // token tiles per row of 256 channels (tile t: tokens t % tiles_m, channels t / tiles_m)
-    int tile0;            // first tile of the launch
-    int sk_tiles;         // 0: one whole tile per CTA; > 0: stream-K over this many tiles
-    float* part;          // stream-K: [gridDim.x][2][kWidePartFloats] partial accumulators
-    uint32_t* arrivals;   // stream-K: [sk_tiles] arrival counts, zero at launch
-};
 
 struct GemmWideCfg {
     static constexpr int kXStages = 4;
@@ -310,36 +292,15 @@ struct GemmWideCfg {
     static constexpr int kAOff = kXOff + kXStages * kXBytes;
     static constexpr int kWOff = kAOff + kABufs * kABytes;
     static constexpr int kBarOff = kWOff + kWStages * kWBytes;
-    static constexpr int kNumBars = 2 * kXStages + 2 * kWStages + 2 * kABufs + 2;
+    static constexpr int kNumBars = 2 * kXStages + 2 * kWStages + 2 * kABufs + 1;
     static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
-    static constexpr int kFlagOff = kTmemPtrOff + 8;
-    static constexpr int kSmemBytes = kFlagOff + 8 + 1024;
+    static constexpr int kSmemBytes = kTmemPtrOff + 16 + 1024;
 };
-
-// The k-block range [xb, xe) of this CTA in the launch's flattened (tile, k-block) space.
-__device__ __forceinline__ void wide_range(const WideSched& w, int nkb, long long& xb, long long& xe) {
-    if (w.sk_tiles == 0) {
-        xb = (long long)blockIdx.x * nkb;
-        xe = xb + nkb;
-    } else {
-        const long long I = (long long)w.sk_tiles * nkb;
-        xb = (long long)blockIdx.x * I / gridDim.x;
-        xe = (long long)(blockIdx.x + 1) * I / gridDim.x;
-    }
-}
-
-// Stream-K: the CTA whose range holds flattened k-block x (the largest c with
-// floor(c I / P) <= x; empty ranges are skipped), and the workspace slot of CTA c's
-// fragment of tile t (0 for the first tile of its range, 1 for the second).
-__device__ __forceinline__ int sk_cta_of(long long x, long long I, int P) { return (int)(((x + 1) * P + I - 1) / I) - 1; }
-__device__ __forceinline__ int sk_slot(int c, int t, long long I, int P, int nkb) {
-    return 2 * c + (t == (int)(((long long)c * I / P) / nkb) ? 0 : 1);
-}
 
 __global__ void __launch_bounds__(kWideThreads, 1)
 gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
                        const uint16_t* __restrict__ scales, const uint32_t* __restrict__ qzeros, int M, int N, int K,
-                       int G, int zero_point, uint16_t* __restrict__ Y, const WideSched sched) {
+                       int G, int zero_point, uint16_t* __restrict__ Y) {
     using C = GemmWideCfg;
     using namespace sm100;
     extern __shared__ uint8_t smem_raw[];
@@ -351,25 +312,14 @@ gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
     uint64_t* wempty = wfull + C::kWStages;         // [kWStages] dequantisers done with it
     uint64_t* afull = wempty + C::kWStages;         // [kABufs]  dequantised tiles written
     uint64_t* aempty = afull + C::kABufs;           // [kABufs]  MMA done with them
-    uint64_t* tfull = aempty + C::kABufs;           // accumulators of a fragment complete
-    uint64_t* tempty = tfull + 1;                   // epilogue done reading them
+    uint64_t* tfull = aempty + C::kABufs;           // accumulators complete
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::kTmemPtrOff);
-    volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kFlagOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * kWideBN;
+    const int n0 = blockIdx.y * kWideRows;
     const int num_kb = ceil_div(K, kGemmKB);
-    long long xb, xe;
-    wide_range(sched, num_kb, xb, xe);
-    // fragment f of the range: tile (relative to tile0) and k-blocks [kb_b, kb_e)
-    auto frag_of = [&](long long x, int& trel, int& kb_b, int& kb_e, int& m0, int& n0) {
-        trel = (int)(x / num_kb);
-        kb_b = (int)(x - (long long)trel * num_kb);
-        kb_e = (int)min((long long)num_kb, (long long)kb_b + (xe - x));
-        const int tile = sched.tile0 + trel;
-        m0 = (tile % sched.tiles_m) * kWideBN;
-        n0 = (tile / sched.tiles_m) * kWideRows;
-    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kXStages; ++s) {
@@ -385,7 +335,6 @@ gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
             mbar_init(&aempty[a], 1);
         }
         mbar_init(tfull, 1);
-        mbar_init(tempty, kDequantWarps);
         mbar_fence_init();
         prefetch_tensormap(&tmap_x);
         prefetch_tensormap(&tmap_q);
@@ -408,66 +357,45 @@ gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
             uint64_t* empty = xs ? xempty : wempty;
             const uint32_t bytes = xs ? C::kXBytes : C::kWBytes;
             uint8_t* base = smem + (xs ? C::kXOff : C::kWOff);
-            int it = 0;
+            int issued = 0;
             bool ok = true;
-            for (long long x = xb; x < xe && ok;) {
-                int trel, kb_b, kb_e, m0, n0;
-                frag_of(x, trel, kb_b, kb_e, m0, n0);
-                for (int kb = kb_b; kb < kb_e; ++kb) {
-                    const int s = it % S;
-                    if (it >= S) ok = mbar_wait(&empty[s], ((it / S) - 1) & 1);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&full[s], bytes);
-                    if (xs)
-                        tma_load_2d(base + s * bytes, &tmap_x, &full[s], kb * kGemmKB, m0);
-                    else
-                        tma_load_2d(base + s * bytes, &tmap_q, &full[s], kb * (kGemmKB / 8), n0);
-                    ++it;
-                }
-                x += kb_e - kb_b;
+            for (int kb = 0; kb < num_kb && ok; ++kb) {
+                const int s = kb % S;
+                if (kb >= S) ok = mbar_wait(&empty[s], ((kb / S) - 1) & 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&full[s], bytes);
+                if (xs)
+                    tma_load_2d(base + s * bytes, &tmap_x, &full[s], kb * kGemmKB, m0);
+                else
+                    tma_load_2d(base + s * bytes, &tmap_q, &full[s], kb * (kGemmKB / 8), n0);
+                ++issued;
             }
-            for (int j = it - 1; j >= 0 && j >= it - S; --j) mbar_wait(&full[j % S], (j / S) & 1);
+            for (int kb = issued - 1; kb >= 0 && kb >= issued - S; --kb) mbar_wait(&full[kb % S], (kb / S) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
             constexpr uint32_t idesc = idesc_f16_f32(kGemmTileN, kWideBN);
-            int it = 0, f = 0;
             bool ok = true;
-            for (long long x = xb; x < xe && ok; ++f) {
-                int trel, kb_b, kb_e, m0, n0;
-                frag_of(x, trel, kb_b, kb_e, m0, n0);
-                if (f > 0) {   // the epilogue has read the previous fragment's accumulators
-                    ok = mbar_wait(tempty, (f - 1) & 1);
-                    if (!ok) break;
-                    tc_fence_after();
-                }
-                for (int kb = kb_b; kb < kb_e; ++kb, ++it) {
-                    const int s = it % C::kXStages;
-                    const int a = it % C::kABufs;
-                    ok = mbar_wait(&xfull[s], (it / C::kXStages) & 1) && mbar_wait(&afull[a], (it / C::kABufs) & 1);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t abase = smem_u32(smem + C::kAOff + a * C::kABytes);
-                    const uint64_t a0 = desc_sw128_kmajor(abase), a1 = desc_sw128_kmajor(abase + C::kATileBytes);
-                    const uint64_t bdesc = desc_sw128_kmajor(smem_u32(smem + C::kXOff + s * C::kXBytes));
-#pragma unroll
-                    for (int kk = 0; kk < kGemmKB / 16; ++kk) {
-                        const uint32_t acc = (kb != kb_b || kk != 0) ? 1u : 0u;
-                        mma_f16(tmem, a0 + 2 * kk, bdesc + 2 * kk, idesc, acc);
-                        mma_f16(tmem + kWideBN, a1 + 2 * kk, bdesc + 2 * kk, idesc, acc);
-                    }
-                    mma_commit(&xempty[s]);
-                    mma_commit(&aempty[a]);
-                }
+            for (int kb = 0; kb < num_kb && ok; ++kb) {
+                const int s = kb % C::kXStages;
+                const int a = kb % C::kABufs;
+                ok = mbar_wait(&xfull[s], (kb / C::kXStages) & 1) && mbar_wait(&afull[a], (kb / C::kABufs) & 1);
                 if (!ok) break;
-                mma_commit(tfull);
-                x += kb_e - kb_b;
+                tc_fence_after();
+                const uint32_t abase = smem_u32(smem + C::kAOff + a * C::kABytes);
+                const uint64_t a0 = desc_sw128_kmajor(abase), a1 = desc_sw128_kmajor(abase + C::kATileBytes);
+                const uint64_t bdesc = desc_sw128_kmajor(smem_u32(smem + C::kXOff + s * C::kXBytes));
+#pragma unroll
+                for (int kk = 0; kk < kGemmKB / 16; ++kk) {
+                    mma_f16(tmem, a0 + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+                    mma_f16(tmem + kWideBN, a1 + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+                }
+                mma_commit(&xempty[s]);
+                mma_commit(&aempty[a]);
             }
-            if (!ok) {   // drain what was issued before TMEM is freed
-                mma_commit(tfull);
-                mbar_wait(tfull, f & 1);
-            }
+            mma_commit(tfull);   // also on the error path, so that the MMAs drain before TMEM is freed
+            if (!ok) mbar_wait(tfull, 0);
         }
     } else {
         // ---------------- dequantise (thread = channel row, 32 codes), then epilogue ----------------
@@ -475,141 +403,82 @@ gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
         const int row = d & (kWideRows - 1);      // 0..255
         const int kh = d >> 8;                    // which 32 channels of the k-block
         const int rt = row >> 7, r = row & 127;
+        const int n = n0 + row;
         const int ng = K / G;
         const int nzw = ceil_div(ng, 8);
         const bool zp = zero_point != 0;
-        // epilogue mapping: TMEM lane quarter q of accumulator ert, token columns t0 .. t0 + 127
-        const int q = warp & 3;
-        const int set = (warp - 3) >> 2;
-        const int ert = set >> 1;
-        const int t0 = (set & 1) * (kWideBN / 2);
-        const int tl = q * 32 + lane;                        // TMEM lane = channel row in the accumulator
-        const uint32_t tcol = (uint32_t)(ert * kWideBN + t0);
-        const long long I = (long long)sched.sk_tiles * num_kb;
-        const int P = gridDim.x;
-        int it = 0, f = 0;
+        const bool row_ok = n < N;
+        const uint16_t* srow = scales + (size_t)(row_ok ? n : 0) * ng;
+        const uint32_t* zrow = qzeros + (size_t)(row_ok ? n : 0) * nzw;
+        int g_next = (kh * 32) / G;
+        uint32_t sc_next = row_ok ? __ldg(srow + g_next) : 0u;
+        uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_next >> 3)) : 0u;
+        int g_cur = -1;
+        uint32_t s2 = 0, zmagic = 0x64006400u, zneg16 = 0;
         bool ok = true;
-        // every fragment runs to its named barriers even after a failed wait (the work is
-        // skipped), so that no warp of the 16 is left waiting on one that stopped
-        for (long long x = xb; x < xe; ++f) {
-            int trel, kb_b, kb_e, m0, n0;
-            frag_of(x, trel, kb_b, kb_e, m0, n0);
-            const int n = n0 + row;
-            const bool row_ok = n < N;
-            const uint16_t* srow = scales + (size_t)(row_ok ? n : 0) * ng;
-            const uint32_t* zrow = qzeros + (size_t)(row_ok ? n : 0) * nzw;
-            int g_next = (kb_b * kGemmKB + kh * 32) / G;
-            uint32_t sc_next = (row_ok && kb_b * kGemmKB + kh * 32 < K) ? __ldg(srow + g_next) : 0u;
-            uint32_t zw_next = (row_ok && zp && kb_b * kGemmKB + kh * 32 < K) ? __ldg(zrow + (g_next >> 3)) : 0u;
-            int g_cur = -1;
-            uint32_t s2 = 0, zmagic = 0x64006400u, zneg16 = 0;
-            for (int kb = kb_b; kb < kb_e && ok; ++kb, ++it) {
-                const int s = it % C::kWStages;
-                const int a = it % C::kABufs;
-                const int k = kb * kGemmKB + kh * 32;
-                const bool live = row_ok && k < K;
-                if (live && g_next != g_cur) {
-                    g_cur = g_next;
-                    const uint32_t sc = sc_next;
-                    const uint32_t z = zp ? ((zw_next >> (4 * (g_cur & 7))) & 15u) : 8u;
-                    s2 = sc | (sc << 16);
-                    const uint32_t zm = 0x6400u | z;
-                    zmagic = zm | (zm << 16);
-                    const uint32_t zn = 0xD000u | (z << 4) | 0x0400u;
-                    zneg16 = zn | (zn << 16);
-                    const float qz_max = zp ? fmaxf((float)z, 15.0f - (float)z) : 8.0f;
-                    if (!(h2f((uint16_t)sc) * qz_max < 65520.0f) && !isnan(h2f((uint16_t)sc))) raise_error(kErrRange);
-                }
-                {   // prefetch the next k-block's group parameters if the group changes
-                    const int kn = k + kGemmKB;
-                    const int gn = kn / G;
-                    if (row_ok && kn < K && gn != g_cur) {
-                        g_next = gn;
-                        sc_next = __ldg(srow + gn);
-                        if (zp) zw_next = __ldg(zrow + (gn >> 3));
-                    }
-                }
-                ok = mbar_wait(&wfull[s], (it / C::kWStages) & 1);
-                if (ok && it >= C::kABufs) ok = mbar_wait(&aempty[a], ((it / C::kABufs) - 1) & 1);
-                if (!ok) break;
-                const uint4 packed =
-                    *reinterpret_cast<const uint4*>(smem + C::kWOff + s * C::kWBytes + row * 32 + kh * 16);
-                uint4 v[4];
-                v[0] = live ? dequant_word(packed.x, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
-                v[1] = live ? dequant_word(packed.y, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
-                v[2] = live ? dequant_word(packed.z, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
-                v[3] = live ? dequant_word(packed.w, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&wempty[s]);     // the packed words are in registers
-                uint8_t* atile = smem + C::kAOff + a * C::kABytes + rt * C::kATileBytes;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(atile + sw128_offset(r, kh * 4 + c)) = v[c];
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&afull[a]);
+        for (int kb = 0; kb < num_kb && ok; ++kb) {
+            const int s = kb % C::kWStages;
+            const int a = kb % C::kABufs;
+            const int k = kb * kGemmKB + kh * 32;
+            const bool live = row_ok && k < K;
+            if (live && g_next != g_cur) {
+                g_cur = g_next;
+                const uint32_t sc = sc_next;
+                const uint32_t z = zp ? ((zw_next >> (4 * (g_cur & 7))) & 15u) : 8u;
+                s2 = sc | (sc << 16);
+                const uint32_t zm = 0x6400u | z;
+                zmagic = zm | (zm << 16);
+                const uint32_t zn = 0xD000u | (z << 4) | 0x0400u;
+                zneg16 = zn | (zn << 16);
+                const float qz_max = zp ? fmaxf((float)z, 15.0f - (float)z) : 8.0f;
+                if (!(h2f((uint16_t)sc) * qz_max < 65520.0f) && !isnan(h2f((uint16_t)sc))) raise_error(kErrRange);
             }
-            // ---- epilogue of the fragment ----
-            if (ok) ok = mbar_wait(tfull, f & 1);
-            tc_fence_after();
-            const bool whole = kb_b == 0 && kb_e == num_kb;
-            const int nn = n0 + ert * kGemmTileN + tl;
-            float* slot = whole ? nullptr : sched.part + ((size_t)blockIdx.x * 2 + f) * kWidePartFloats;
-            for (int c = 0; c < kWideBN / 2 && ok; c += 16) {
-                uint32_t rv[16];
-                tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + tcol + (uint32_t)c, rv);
-                tmem_ld_wait();
-                if (whole) {
-                    if (nn < N) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int m = m0 + t0 + c + j;
-                            if (m < M) Y[(size_t)m * N + nn] = f2h_rn(__uint_as_float(rv[j]));
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) slot[(size_t)(tcol + c + j) * kGemmTileN + tl] = __uint_as_float(rv[j]);
+            {   // prefetch the next k-block's group parameters if the group changes
+                const int kn = k + kGemmKB;
+                const int gn = kn / G;
+                if (row_ok && kn < K && gn != g_cur) {
+                    g_next = gn;
+                    sc_next = __ldg(srow + gn);
+                    if (zp) zw_next = __ldg(zrow + (gn >> 3));
                 }
             }
-            tc_fence_before();
+            ok = mbar_wait(&wfull[s], (kb / C::kWStages) & 1);
+            if (ok && kb >= C::kABufs) ok = mbar_wait(&aempty[a], ((kb / C::kABufs) - 1) & 1);
+            if (!ok) break;
+            const uint4 packed = *reinterpret_cast<const uint4*>(smem + C::kWOff + s * C::kWBytes + row * 32 + kh * 16);
+            uint4 v[4];
+            v[0] = live ? dequant_word(packed.x, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+            v[1] = live ? dequant_word(packed.y, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+            v[2] = live ? dequant_word(packed.z, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+            v[3] = live ? dequant_word(packed.w, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty);
-            if (!whole) {
-                // count this contribution; the last of the tile's contributors adds them up
-                __threadfence();
-                asm volatile("bar.sync 1, %0;" ::"n"(kDequantWarps * 32) : "memory");
-                if (d == 0) {
-                    const int c_first = sk_cta_of((long long)trel * num_kb, I, P);
-                    const int c_last = sk_cta_of((long long)(trel + 1) * num_kb - 1, I, P);
-                    const uint32_t old = ok ? atomicAdd(sched.arrivals + trel, 1u) : 0u;
-                    *last_flag = (ok && old + 1u == (uint32_t)(c_last - c_first + 1)) ? 1u : 0u;
-                }
-                asm volatile("bar.sync 1, %0;" ::"n"(kDequantWarps * 32) : "memory");
-                if (*last_flag) {
-                    __threadfence();
-                    const int c_first = sk_cta_of((long long)trel * num_kb, I, P);
-                    const int c_last = sk_cta_of((long long)(trel + 1) * num_kb - 1, I, P);
-                    for (int c = 0; c < kWideBN / 2; c += 16) {
-                        float acc[16];
+            if (lane == 0) mbar_arrive(&wempty[s]);     // the packed words are in registers
+            uint8_t* atile = smem + C::kAOff + a * C::kABytes + rt * C::kATileBytes;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-                        for (int cc = c_first; cc <= c_last; ++cc) {
-                            const float* src = sched.part + (size_t)sk_slot(cc, trel, I, P, num_kb) * kWidePartFloats;
+            for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(atile + sw128_offset(r, kh * 4 + c)) = v[c];
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[a]);
+        }
+        if (ok && mbar_wait(tfull, 0)) {
+            tc_fence_after();
+            const int q = warp & 3;                        // TMEM lane quarter this warp may access
+            const int set = (warp - 3) >> 2;               // 0..3: four warps per lane quarter
+            const int ert = set >> 1;                      // accumulator (row tile) of this set
+            const int t0 = (set & 1) * (kWideBN / 2);      // its 128 token columns
+            const int nn = n0 + ert * kGemmTileN + q * 32 + lane;
+            for (int c = 0; c < kWideBN / 2; c += 16) {
+                uint32_t rv[16];
+                tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ert * kWideBN + t0 + c), rv);
+                tmem_ld_wait();
+                if (nn < N) {
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) acc[j] += __ldcg(src + (size_t)(tcol + c + j) * kGemmTileN + tl);
-                        }
-                        if (nn < N) {
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const int m = m0 + t0 + c + j;
-                                if (m < M) Y[(size_t)m * N + nn] = f2h_rn(acc[j]);
-                            }
-                        }
+                    for (int j = 0; j < 16; ++j) {
+                        const int m = m0 + t0 + c + j;
+                        if (m < M) Y[(size_t)m * N + nn] = f2h_rn(__uint_as_float(rv[j]));
                     }
-                    if (d == 0) sched.arrivals[trel] = 0u;   // ready for the next launch
                 }
             }
-            x += kb_e - kb_b;
         }
     }
     tc_fence_before();
@@ -722,55 +591,15 @@ inline int gemm_splits(int M, int N, int K, int sms) {
     return std::max(1, s);
 }
 
-// Tiles of the wide form: whole waves data-parallel; the tiles of a last, partial wave
-// (when there is more than one wave) stream-K over min(sms, 4 x those tiles) CTAs, each
-// taking an equal share of their k-blocks (at least 4 k-blocks each on average).
-struct WidePlan {
-    int tiles_m;   // token tiles
-    int dp;        // tiles launched one per CTA
-    int sk;        // tiles shared by stream-K
-    int sk_ctas;   // CTAs of the stream-K launch
-};
-
-inline WidePlan wide_plan(int M, int N, int K, int sms) {
-    WidePlan p = {};
-    p.tiles_m = ceil_div(M, kWideBN);
-    const long long tiles = (long long)p.tiles_m * ceil_div(N, kWideRows);
-    const int rem = (int)(tiles % sms);
-    const int num_kb = ceil_div(K, kGemmKB);
-    p.dp = (int)tiles;
-    if (tiles > sms && rem > 0) {
-        const int ctas = std::min(sms, std::min(4 * rem, (int)(((long long)rem * num_kb) / 4)));
-        if (ctas > rem) {
-            p.sk = rem;
-            p.dp = (int)(tiles - rem);
-            p.sk_ctas = ctas;
-        }
-    }
-    return p;
-}
-
-// Stream-K scratch: the arrival counts (one word per tile), then two partial
-// accumulators per CTA.
-inline size_t wide_sk_bytes(const WidePlan& p) {
-    if (p.sk == 0) return 0;
-    return align256((size_t)p.sk * 4) + (size_t)p.sk_ctas * 2 * kWidePartFloats * 4;
-}
-
-inline bool use_wide_gemm(int M, int N, int sms);
-
-// Workspace of the GEMM: the fp32 partial sums of the split-K form, or the stream-K
-// scratch of the wide form (0 when neither is used).
+// Workspace of the GEMM: the fp32 partial sums of the split-K form (0 when it is not used).
 inline size_t gemm_workspace_bytes(int M, int N, int K, int sms) {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
-    if (use_wide_gemm(M, N, sms)) return wide_sk_bytes(wide_plan(M, N, K, sms));
     const int s = gemm_splits(M, N, K, sms);
     return s > 1 ? (size_t)s * M * N * 4 : 0;
 }
 
 inline awq_status launch_gemm_wide(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
-                                   const uint32_t* qzeros, int N, int K, int G, int zp, uint16_t* Y, cudaStream_t st,
-                                   int sms, void* ws, size_t ws_bytes) {
+                                   const uint32_t* qzeros, int N, int K, int G, int zp, uint16_t* Y, cudaStream_t st) {
     using C = GemmWideCfg;
     CUtensorMap tx, tq;
     if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)M, (uint64_t)K, kWideBN, kGemmKB,
@@ -782,25 +611,9 @@ inline awq_status launch_gemm_wide(const uint16_t* X, int M, const uint32_t* qwe
     if (cudaFuncSetAttribute(gemm_w4a16_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
         return AWQ_ERR_CUDA;
-    WidePlan p = wide_plan(M, N, K, sms);
-    const size_t need = wide_sk_bytes(p);
-    if (need > 0 && (ws == nullptr || ws_bytes < need)) {   // no scratch: every tile data-parallel
-        p.dp += p.sk;
-        p.sk = 0;
-    }
-    WideSched sc = {p.tiles_m, 0, 0, nullptr, nullptr};
-    if (p.dp > 0)
-        gemm_w4a16_wide_kernel<<<p.dp, kWideThreads, C::kSmemBytes, st>>>(tx, tq, scales, qzeros, M, N, K, G, zp, Y,
-                                                                           sc);
-    if (p.sk > 0) {
-        sc.tile0 = p.dp;
-        sc.sk_tiles = p.sk;
-        sc.arrivals = static_cast<uint32_t*>(ws);
-        sc.part = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)p.sk * 4));
-        if (cudaMemsetAsync(sc.arrivals, 0, (size_t)p.sk * 4, st) != cudaSuccess) return AWQ_ERR_CUDA;
-        gemm_w4a16_wide_kernel<<<p.sk_ctas, kWideThreads, C::kSmemBytes, st>>>(tx, tq, scales, qzeros, M, N, K, G,
-                                                                                zp, Y, sc);
-    }
+    dim3 grid(ceil_div(M, kWideBN), ceil_div(N, kWideRows));
+    if (grid.y > 65535u) return AWQ_ERR_UNSUPPORTED;
+    gemm_w4a16_wide_kernel<<<grid, kWideThreads, C::kSmemBytes, st>>>(tx, tq, scales, qzeros, M, N, K, G, zp, Y);
     return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
@@ -821,8 +634,7 @@ inline bool use_wide_gemm(int M, int N, int sms) {
 inline awq_status launch_gemm_w4a16(const uint16_t* X, int M, const uint32_t* qweight, const uint16_t* scales,
                                     const uint32_t* qzeros, int N, int K, int G, int zp, uint16_t* Y, cudaStream_t st,
                                     int sms, void* ws, size_t ws_bytes) {
-    if (use_wide_gemm(M, N, sms))
-        return launch_gemm_wide(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st, sms, ws, ws_bytes);
+    if (use_wide_gemm(M, N, sms)) return launch_gemm_wide(X, M, qweight, scales, qzeros, N, K, G, zp, Y, st);
     // split K over the caller's workspace when the tiles alone leave SMs idle (as many
     // splits as the workspace holds, up to the chosen number)
     int splits = gemm_splits(M, N, K, sms);

@@ -205,17 +205,11 @@ awq_status awq_linear_gemv(const uint16_t* X, int32_t M, const uint32_t* qweight
  * awq_linear_gemv; the weight tile is dequantised to fp16 ((q-zero)*scale16,
  * one rounding) in shared memory and multiplied on the tcgen05 tensor cores with
  * fp32 accumulation in tensor memory.  Any M >= 1.
- * Workspace (awq_workspace_bytes(AWQ_OP_GEMM, ...)): when the batch gives fewer
- * 128-channel tiles than the GPU has SMs, the kernel splits K into up to ws_bytes /
- * (4 M N) parts whose fp32 partial sums go to ws and are added in a fixed order into Y
- * (one fp16 rounding).  For prefill batches (256 x 256 tiles) whose tiles fill more than
- * one wave of SMs and leave the last wave partly empty, the tiles of that last wave are
- * shared out in equal ranges of k-blocks over the SMs instead: each share's fp32
- * accumulator and one arrival count per tile go to ws, and the last share of a tile to
- * finish adds them in k order into Y.  ws may be NULL (or small), which only disables
- * these forms.  The result depends on which form runs (the fp32 addition order), and so
- * on the SM count, but is the same on every run of one device.  ws must not be used by
- * two calls at once.
+ * Workspace: when the batch gives fewer 128-channel tiles than the GPU has SMs, the
+ * kernel splits K into up to awq_workspace_bytes(AWQ_OP_GEMM, ...) / (4 M N) parts whose
+ * fp32 partial sums go to ws and are added in a fixed order into Y (one fp16 rounding);
+ * ws may be NULL (or small), which only disables the split.  ws must not be used by two
+ * calls at once.
  * Range: each dequantised weight is rounded once to fp16, so it must be finite there:
  * max|q - zero| * scale16 < 65520 for every group (max|q - zero| is max(zero, 15 - zero),
  * or 8 without zero point).  awq_quantize_pack gives that whenever the group's scaled

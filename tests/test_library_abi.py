@@ -101,12 +101,8 @@ def test_scale_search_argument_errors(lib):
 def test_workspace_sizes(lib):
     assert lib.awq_workspace_bytes(0, 1, 4096, 4096, _cfg()) == 0
     assert lib.awq_workspace_bytes(2, 1, 4096, 4096, _cfg()) == 0
-    # the GEMM needs a workspace only where its tiles leave SMs idle (148 SMs without a
-    # device): whole waves of 256 x 256 prefill tiles need none (8 x 37 = 2 x 148) ...
-    assert lib.awq_workspace_bytes(3, 2048, 37 * 256, 8192, _cfg()) == 0
-    # ... a last wave of 108 tiles is shared by 148 CTAs: 108 arrival words (256-byte
-    # aligned), then two fp32 accumulators of 512 x 128 per CTA
-    assert lib.awq_workspace_bytes(3, 2048, 8192, 8192, _cfg()) == 512 + 148 * 2 * 512 * 128 * 4
+    # the GEMM needs a workspace only to split K when its tiles leave SMs idle
+    assert lib.awq_workspace_bytes(3, 2048, 8192, 8192, _cfg()) == 0
     small = lib.awq_workspace_bytes(3, 16, 4096, 4096, _cfg())
     assert small > 0 and small % (16 * 4096 * 4) == 0
     a = lib.awq_workspace_bytes(1, 512, 4096, 4096, _cfg())

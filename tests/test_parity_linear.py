@@ -187,13 +187,11 @@ def test_gemm_llama70b_prefill_sampled(lib):
         assert_linear_close(y[:, rows], ref)
 
 
-def test_gemm_stream_k_last_wave(lib):
-    """A prefill shape whose 256 x 256 tiles fill one wave of 148 SMs and 12 tiles of a
-    second: those 12 tiles' k-blocks are shared by 33 CTAs of 4 k-blocks each (3 or 4
-    per tile; ragged M and N), the last CTA of a tile to finish adding the partial sums.
-    Every output channel of the shared tiles and a sample of the rest against the
-    oracle; a second call gives the same bits (the arrival counts start from zero again);
-    without a workspace every tile runs whole, also within the rule."""
+def test_gemm_wide_two_waves_ragged(lib):
+    """A prefill shape on the wide form with more 256 x 256 tiles (160) than one wave of
+    SMs, ragged in M (300 tokens) and N (20440 channels): every output channel of the last
+    7 channel tiles and a sample of the rest against the oracle, and a second call gives
+    the same bits."""
     M, K, N, G = 300, 704, 20440, 64
     W = inputs.weights(N, K, 0.02, seed=320)
     X = inputs.activations(M, K, seed=321)
@@ -205,12 +203,7 @@ def test_gemm_stream_k_last_wave(lib):
     assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
     rng = np.random.Generator(np.random.PCG64(322))
     rows = np.concatenate([np.sort(rng.choice(74 * 256, 96, replace=False)), np.arange(74 * 256, N)])
-    ref = O.linear_rows(X, q, sc, z, K, G, True, rows)
-    assert_linear_close(y1[:, rows], ref)
-    tiny = torch.empty(16, dtype=torch.uint8, device="cuda")
-    y3 = to_np(lib.linear_gemm(Xd, dq[0], dq[1], dq[2], G, True, workspace=tiny))
-    lib.device_error()
-    assert_linear_close(y3[:, rows], ref)
+    assert_linear_close(y1[:, rows], O.linear_rows(X, q, sc, z, K, G, True, rows))
 
 
 def _edge_weights(K):
