@@ -181,9 +181,9 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         const uint32_t* zrow = qzeros + (size_t)(row_ok ? n : 0) * nzw;
         // scale and zero word of the thread's group, loaded one k-block ahead (raw; using a
         // loaded value stalls on its load) and only when the group changes
-        int g_next = (kb0 * kGemmKB + kq * 16) / G;
-        uint32_t sc_next = row_ok ? __ldg(srow + g_next) : 0u;
-        uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_next >> 3)) : 0u;
+        const int g_first = (kb0 * kGemmKB + kq * 16) / G;
+        uint32_t sc_next = row_ok ? __ldg(srow + g_first) : 0u;
+        uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_first >> 3)) : 0u;
         int g_cur = -1;
         uint32_t s2 = 0, zmagic = 0x64006400u, zneg16 = 0;
         bool ok = true;
@@ -192,8 +192,9 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
             const int a = kb % C::kABufs;
             const int k = (kb0 + kb) * kGemmKB + kq * 16;
             const bool live = row_ok && k < K;
-            if (live && g_next != g_cur) {
-                g_cur = g_next;
+            const int g_here = k / G;
+            if (live && g_here != g_cur) {   // sc_next / zw_next hold this group's parameters
+                g_cur = g_here;
                 const uint32_t sc = sc_next;
                 const uint32_t z = zp ? ((zw_next >> (4 * (g_cur & 7))) & 15u) : 8u;
                 s2 = sc | (sc << 16);
@@ -205,12 +206,10 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                 // iff max|q - z| * scale16 < 65520 (exact in fp32); otherwise flag it
                 const float qz_max = zp ? fmaxf((float)z, 15.0f - (float)z) : 8.0f;
                 if (!(h2f((uint16_t)sc) * qz_max < 65520.0f) && !isnan(h2f((uint16_t)sc))) raise_error(kErrRange);
-            }
-            {   // prefetch the next k-block's group parameters if the group changes
-                const int kn = k + kGemmKB;
-                const int gn = kn / G;
-                if (row_ok && kn < K && gn != g_cur) {
-                    g_next = gn;
+                // the next group this thread reaches (G / 64 k-blocks on, at least one): its
+                // parameters are fetched now, a whole group ahead of their use
+                const int gn = g_cur + (G >= kGemmKB ? 1 : kGemmKB / G);
+                if (gn * G < K) {
                     sc_next = __ldg(srow + gn);
                     if (zp) zw_next = __ldg(zrow + (gn >> 3));
                 }
@@ -410,9 +409,9 @@ gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
         const bool row_ok = n < N;
         const uint16_t* srow = scales + (size_t)(row_ok ? n : 0) * ng;
         const uint32_t* zrow = qzeros + (size_t)(row_ok ? n : 0) * nzw;
-        int g_next = (kh * 32) / G;
-        uint32_t sc_next = row_ok ? __ldg(srow + g_next) : 0u;
-        uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_next >> 3)) : 0u;
+        const int g_first = (kh * 32) / G;
+        uint32_t sc_next = row_ok ? __ldg(srow + g_first) : 0u;
+        uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_first >> 3)) : 0u;
         int g_cur = -1;
         uint32_t s2 = 0, zmagic = 0x64006400u, zneg16 = 0;
         bool ok = true;
@@ -421,8 +420,9 @@ gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
             const int a = kb % C::kABufs;
             const int k = kb * kGemmKB + kh * 32;
             const bool live = row_ok && k < K;
-            if (live && g_next != g_cur) {
-                g_cur = g_next;
+            const int g_here = k / G;
+            if (live && g_here != g_cur) {   // sc_next / zw_next hold this group's parameters
+                g_cur = g_here;
                 const uint32_t sc = sc_next;
                 const uint32_t z = zp ? ((zw_next >> (4 * (g_cur & 7))) & 15u) : 8u;
                 s2 = sc | (sc << 16);
@@ -432,12 +432,10 @@ gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
                 zneg16 = zn | (zn << 16);
                 const float qz_max = zp ? fmaxf((float)z, 15.0f - (float)z) : 8.0f;
                 if (!(h2f((uint16_t)sc) * qz_max < 65520.0f) && !isnan(h2f((uint16_t)sc))) raise_error(kErrRange);
-            }
-            {   // prefetch the next k-block's group parameters if the group changes
-                const int kn = k + kGemmKB;
-                const int gn = kn / G;
-                if (row_ok && kn < K && gn != g_cur) {
-                    g_next = gn;
+                // the next group this thread reaches (G / 64 k-blocks on, at least one): its
+                // parameters are fetched now, a whole group ahead of their use
+                const int gn = g_cur + (G >= kGemmKB ? 1 : kGemmKB / G);
+                if (gn * G < K) {
                     sc_next = __ldg(srow + gn);
                     if (zp) zw_next = __ldg(zrow + (gn >> 3));
                 }
