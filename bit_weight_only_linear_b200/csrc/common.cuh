@@ -38,6 +38,19 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+
+// Largest / smallest of three floats, one instruction each on sm_100 (the three-operand
+// forms of max.f32 / min.f32; a NaN operand is ignored as in fmaxf / fminf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 __device__ __forceinline__ uint16_t f2h_rn(float f) { return __half_as_ushort(__float2half_rn(f)); }
 
 // Correctly rounded double -> binary16 (one rounding, nearest-even), by the

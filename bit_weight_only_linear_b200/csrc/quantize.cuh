@@ -194,11 +194,11 @@ quantize_pack_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict_
         mul_f16x2_f32(wv[r].y, sv.y, ws[r][2], ws[r][3]);
         mul_f16x2_f32(wv[r].z, sv.z, ws[r][4], ws[r][5]);
         mul_f16x2_f32(wv[r].w, sv.w, ws[r][6], ws[r][7]);
-        float mx = ws[r][0], mn = ws[r][0];
+        float mx = fmaxf(ws[r][0], ws[r][1]), mn = fminf(ws[r][0], ws[r][1]);
 #pragma unroll
-        for (int i = 1; i < 8; ++i) {
-            mx = fmaxf(mx, ws[r][i]);
-            mn = fminf(mn, ws[r][i]);
+        for (int i = 2; i < 8; i += 2) {
+            mx = fmax3(mx, ws[r][i], ws[r][i + 1]);
+            mn = fmin3(mn, ws[r][i], ws[r][i + 1]);
         }
 #pragma unroll
         for (int off = (G >> 3) >> 1; off > 0; off >>= 1) {

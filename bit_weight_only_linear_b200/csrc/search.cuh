@@ -356,8 +356,8 @@ search_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* 
                     for (int h = 0; h < 8; ++h) {
                         float a, b;
                         mul_f16x2_f32(wpk[j][h], sw[h], a, b);                  // W s, exact
-                        mx = fmaxf(mx, fmaxf(a, b));
-                        mn = fminf(mn, fminf(a, b));
+                        mx = fmax3(mx, a, b);
+                        mn = fmin3(mn, a, b);
                     }
                 } else {
                     mx = fmaxf(mx, 0.0f);
