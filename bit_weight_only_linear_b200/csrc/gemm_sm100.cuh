@@ -40,7 +40,11 @@ constexpr int kDequantThreads = kDequantWarps * 32;   // 4 threads per row, 16 c
 template <int BN>
 struct GemmCfg {
     static constexpr int kStages = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
-    static constexpr int kABufs = BN >= 256 ? 3 : 4;
+    static constexpr int kABufs = BN >= 256 ? 3 : (BN >= 128 ? 4 : 8);
+    // k-blocks a dequantising thread converts per iteration (one fence and one wait per
+    // barrier round trip for all of them); half the A buffers, so that the MMA consumes
+    // one batch while the next is written
+    static constexpr int kBatch = BN >= 256 ? 1 : kABufs / 2;
     static constexpr int kXBytes = BN * 128;                 // X tile: BN rows x 128 B
     static constexpr int kWBytes = kGemmTileN * 32;          // packed tile: 128 rows x 32 B
     static constexpr int kABytes = kGemmTileN * 128;         // dequantised tile
@@ -52,6 +56,7 @@ struct GemmCfg {
     static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kTmemPtrOff + 16 + 1024;   // + slack to align the base to 1024
     static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+    static_assert(kSmemBytes <= 232448, "shared memory of one CTA exceeds 227 KB");
 };
 
 // (q - z) * s for the 8 codes of one word, returned as 4 fp16 pairs in k order.  The
@@ -187,46 +192,62 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         int g_cur = -1;
         uint32_t s2 = 0, zmagic = 0x64006400u, zneg16 = 0;
         bool ok = true;
-        for (int kb = 0; kb < num_kb && ok; ++kb) {
-            const int s = kb % C::kStages;
-            const int a = kb % C::kABufs;
-            const int k = (kb0 + kb) * kGemmKB + kq * 16;
-            const bool live = row_ok && k < K;
-            const int g_here = k / G;
-            if (live && g_here != g_cur) {   // sc_next / zw_next hold this group's parameters
-                g_cur = g_here;
-                const uint32_t sc = sc_next;
-                const uint32_t z = zp ? ((zw_next >> (4 * (g_cur & 7))) & 15u) : 8u;
-                s2 = sc | (sc << 16);
-                const uint32_t zm = 0x6400u | z;                                   // 1024 + z
-                zmagic = zm | (zm << 16);
-                const uint32_t zn = 0xD000u | (z << 4) | 0x0400u;                  // fp16 -(64 + z): 2^6 * (1 + z/64)
-                zneg16 = zn | (zn << 16);
-                // the fp16 product (q - z) * scale16 is finite for every code of the group
-                // iff max|q - z| * scale16 < 65520 (exact in fp32); otherwise flag it
-                const float qz_max = zp ? fmaxf((float)z, 15.0f - (float)z) : 8.0f;
-                if (!(h2f((uint16_t)sc) * qz_max < 65520.0f) && !isnan(h2f((uint16_t)sc))) raise_error(kErrRange);
-                // the next group this thread reaches (G / 64 k-blocks on, at least one): its
-                // parameters are fetched now, a whole group ahead of their use
-                const int gn = g_cur + (G >= kGemmKB ? 1 : kGemmKB / G);
-                if (gn * G < K) {
-                    sc_next = __ldg(srow + gn);
-                    if (zp) zw_next = __ldg(zrow + (gn >> 3));
+        constexpr int D = C::kBatch;
+        for (int kb = 0; kb < num_kb && ok; kb += D) {
+            // the batch's A buffers free and its packed tiles landed
+#pragma unroll
+            for (int i = 0; i < D; ++i) {
+                const int kbi = kb + i;
+                if (kbi < num_kb) {
+                    if (kbi >= C::kABufs) ok = ok && mbar_wait(&aempty[kbi % C::kABufs], ((kbi / C::kABufs) - 1) & 1);
+                    ok = ok && mbar_wait(&full[kbi % C::kStages], (kbi / C::kStages) & 1);
                 }
             }
-            if (kb >= C::kABufs) ok = mbar_wait(&aempty[a], ((kb / C::kABufs) - 1) & 1);
-            ok = ok && mbar_wait(&full[s], (kb / C::kStages) & 1);
             if (!ok) break;
-            const uint2 packed =
-                *reinterpret_cast<const uint2*>(smem + C::kWOff + s * C::kWBytes + row * 32 + kq * 8);
-            uint8_t* atile = smem + C::kAOff + a * C::kABytes;
-            const uint4 v0 = live ? dequant_word(packed.x, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
-            const uint4 v1 = live ? dequant_word(packed.y, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(atile + sw128_offset(row, kq * 2)) = v0;
-            *reinterpret_cast<uint4*>(atile + sw128_offset(row, kq * 2 + 1)) = v1;
+#pragma unroll
+            for (int i = 0; i < D; ++i) {
+                const int kbi = kb + i;
+                if (kbi >= num_kb) break;
+                const int k = (kb0 + kbi) * kGemmKB + kq * 16;
+                const bool live = row_ok && k < K;
+                const int g_here = k / G;
+                if (live && g_here != g_cur) {   // sc_next / zw_next hold this group's parameters
+                    g_cur = g_here;
+                    const uint32_t sc = sc_next;
+                    const uint32_t z = zp ? ((zw_next >> (4 * (g_cur & 7))) & 15u) : 8u;
+                    s2 = sc | (sc << 16);
+                    const uint32_t zm = 0x6400u | z;                               // 1024 + z
+                    zmagic = zm | (zm << 16);
+                    const uint32_t zn = 0xD000u | (z << 4) | 0x0400u;              // fp16 -(64 + z): 2^6 * (1 + z/64)
+                    zneg16 = zn | (zn << 16);
+                    // the fp16 product (q - z) * scale16 is finite for every code of the group
+                    // iff max|q - z| * scale16 < 65520 (exact in fp32); otherwise flag it
+                    const float qz_max = zp ? fmaxf((float)z, 15.0f - (float)z) : 8.0f;
+                    if (!(h2f((uint16_t)sc) * qz_max < 65520.0f) && !isnan(h2f((uint16_t)sc))) raise_error(kErrRange);
+                    // the next group this thread reaches (G / 64 k-blocks on, at least one): its
+                    // parameters are fetched now, a whole group ahead of their use
+                    const int gn = g_cur + (G >= kGemmKB ? 1 : kGemmKB / G);
+                    if (gn * G < K) {
+                        sc_next = __ldg(srow + gn);
+                        if (zp) zw_next = __ldg(zrow + (gn >> 3));
+                    }
+                }
+                const int s = kbi % C::kStages;
+                const uint2 packed =
+                    *reinterpret_cast<const uint2*>(smem + C::kWOff + s * C::kWBytes + row * 32 + kq * 8);
+                uint8_t* atile = smem + C::kAOff + (kbi % C::kABufs) * C::kABytes;
+                const uint4 v0 = live ? dequant_word(packed.x, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+                const uint4 v1 = live ? dequant_word(packed.y, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(atile + sw128_offset(row, kq * 2)) = v0;
+                *reinterpret_cast<uint4*>(atile + sw128_offset(row, kq * 2 + 1)) = v1;
+            }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&afull[a]);
+            if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < D; ++i)
+                    if (kb + i < num_kb) mbar_arrive(&afull[(kb + i) % C::kABufs]);
+            }
         }
         if (ok && mbar_wait(tfull, 0)) {
             tc_fence_after();
@@ -577,16 +598,24 @@ awq_status launch_gemm_bn(const uint16_t* X, int M, const uint32_t* qweight, con
     return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
-// K splits of the 128-channel form for a batch whose tiles leave SMs idle: enough splits
-// for about two CTAs per SM, each split at least 4 k-blocks (256 channels).  1 = none.
+// K splits of the 128-channel form for a batch whose tiles leave SMs idle (one CTA per
+// SM).  Model of a split's time: a fixed start (TMA round trips, TMEM, the epilogue;
+// about 3000 cycles) plus its k-blocks (about 400 cycles each with batched
+// dequantisation), times the waves the CTAs take; the split count minimising it, each
+// split at least 4 k-blocks, at most 16 splits.  1 = none.
 inline int gemm_splits(int M, int N, int K, int sms) {
     const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
     const long long tiles = (long long)ceil_div(M, bn) * ceil_div(N, kGemmTileN);
     const int num_kb = ceil_div(K, kGemmKB);
     if (tiles >= sms) return 1;
-    int s = (int)((2LL * sms + tiles - 1) / tiles);
-    s = std::min(s, std::max(1, num_kb / 4));
-    return std::max(1, s);
+    int best = 1;
+    double best_t = 1e300;
+    for (int s = 1; s <= 16 && s <= std::max(1, num_kb / 4); ++s) {
+        const double waves = (double)((tiles * s + sms - 1) / sms);
+        const double t = waves * (3000.0 + 400.0 * ceil_div(num_kb, s));
+        if (t < best_t * 0.999) best_t = t, best = s;
+    }
+    return best;
 }
 
 // Workspace of the GEMM: the fp32 partial sums of the split-K form (0 when it is not used).
