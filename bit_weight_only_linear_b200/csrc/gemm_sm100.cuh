@@ -11,14 +11,18 @@
 // is dequantised once per CTA and reused for BN tokens, so the dequant work per
 // multiply-add is 1/BN, and small token counts use a narrow MMA instead of padding.
 //
-// Warp roles (576 threads):
-//   warp 0      TMA producer: X tile [BN x 64] fp16 (128B swizzle) and the packed
-//               weight tile [128 x 8 words] per 64-channel k-block, into an S-stage ring.
+// Warp roles (608 threads):
+//   warp 0      TMA producer of X: tile [BN x 64] fp16 (128B swizzle) per 64-channel k-block,
+//               into a ring whose slots the MMAs free.
 //   warp 1      allocates TMEM; one lane issues 4 tcgen05.mma (K = 16 each) per k-block.
-//   warps 2..17 dequantise: thread (row, quarter) turns 16 codes into fp16
-//               (q - z) * scale16 with mask/magic-number arithmetic and writes them in
-//               the 128B-swizzled K-major layout the MMA reads; afterwards they are the
-//               epilogue, reading the fp32 accumulator from TMEM and storing fp16 Y.
+//   warp 2      TMA producer of the packed weights: tile [128 x 8 words] per k-block, into a
+//               ring of its own whose slots the dequantisers free as soon as they have read
+//               the words, so that refilling it never waits for the MMAs.
+//   warps 3..18 dequantise: thread (row, quarter) turns 16 codes per k-block into fp16
+//               (q - z) * scale16 with mask/magic-number arithmetic, a batch of k-blocks per
+//               iteration, and writes them in the 128B-swizzled K-major layout the MMA
+//               reads; afterwards they are the epilogue, reading the fp32 accumulator from
+//               TMEM and storing fp16 Y (or fp32 partial sums of a K split).
 // Every wait is bounded (2 s): on time-out the kernel raises the device error word,
 // drains what it issued, frees TMEM and returns.
 #pragma once
@@ -32,15 +36,17 @@
 namespace awq {
 
 constexpr int kDequantWarps = 16;
-constexpr int kGemmThreads = 64 + kDequantWarps * 32;   // TMA warp, MMA warp, dequant/epilogue warps
+constexpr int kGemmThreads = 96 + kDequantWarps * 32;   // X TMA, MMA, W TMA, dequant/epilogue warps
 constexpr int kGemmTileN = 128;      // output channels per CTA (MMA M)
 constexpr int kGemmKB = 64;          // input channels per k-block
 constexpr int kDequantThreads = kDequantWarps * 32;   // 4 threads per row, 16 codes each
 
 template <int BN>
 struct GemmCfg {
-    static constexpr int kStages = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
-    static constexpr int kABufs = BN >= 256 ? 3 : (BN >= 128 ? 4 : 8);
+    static constexpr int kXStages = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
+    // packed weights: deep enough to keep a DRAM round trip in flight
+    static constexpr int kWStages = BN >= 256 ? 4 : (BN >= 128 ? 8 : (BN >= 64 ? 12 : 16));
+    static constexpr int kABufs = BN >= 256 ? 3 : (BN >= 128 ? 4 : (BN >= 64 ? 6 : 8));
     // k-blocks a dequantising thread converts per iteration (one fence and one wait per
     // barrier round trip for all of them); half the A buffers, so that the MMA consumes
     // one batch while the next is written
@@ -49,14 +55,15 @@ struct GemmCfg {
     static constexpr int kWBytes = kGemmTileN * 32;          // packed tile: 128 rows x 32 B
     static constexpr int kABytes = kGemmTileN * 128;         // dequantised tile
     static constexpr int kXOff = 0;
-    static constexpr int kAOff = kXOff + kStages * kXBytes;  // both multiples of 1024
+    static constexpr int kAOff = kXOff + kXStages * kXBytes;  // both multiples of 1024
     static constexpr int kWOff = kAOff + kABufs * kABytes;
-    static constexpr int kBarOff = kWOff + kStages * kWBytes;
-    static constexpr int kNumBars = 2 * kStages + 2 * kABufs + 1;
+    static constexpr int kBarOff = kWOff + kWStages * kWBytes;
+    static constexpr int kNumBars = 2 * kXStages + 2 * kWStages + 2 * kABufs + 1;
     static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kTmemPtrOff + 16 + 1024;   // + slack to align the base to 1024
     static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
     static_assert(kSmemBytes <= 232448, "shared memory of one CTA exceeds 227 KB");
+    static_assert(kWStages >= kBatch && kXStages >= kBatch && kABufs >= 2 * kBatch || kBatch == 1, "ring depths");
 };
 
 // (q - z) * s for the 8 codes of one word, returned as 4 fp16 pairs in k order.  The
@@ -93,9 +100,11 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-    uint64_t* full = bars;                          // [kStages]  TMA landed
-    uint64_t* empty = bars + C::kStages;            // [kStages]  MMA done with the X / packed slot
-    uint64_t* afull = empty + C::kStages;           // [kABufs]   dequantised tile written
+    uint64_t* xfull = bars;                         // [kXStages] X landed
+    uint64_t* xempty = xfull + C::kXStages;         // [kXStages] MMA done with the X slot
+    uint64_t* wfull = xempty + C::kXStages;         // [kWStages] packed tile landed
+    uint64_t* wempty = wfull + C::kWStages;         // [kWStages] dequantisers have read it
+    uint64_t* afull = wempty + C::kWStages;         // [kABufs]   dequantised tile written
     uint64_t* aempty = afull + C::kABufs;           // [kABufs]   MMA done with the dequantised tile
     uint64_t* tfull = aempty + C::kABufs;           // accumulator complete
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::kTmemPtrOff);
@@ -110,12 +119,16 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
     const int num_kb = max(0, min(kb_per, ceil_div(K, kGemmKB) - kb0));
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < C::kXStages; ++s) {
+            mbar_init(&xfull[s], 1);
+            mbar_init(&xempty[s], 1);
+        }
+        for (int s = 0; s < C::kWStages; ++s) {
+            mbar_init(&wfull[s], 1);
+            mbar_init(&wempty[s], kDequantWarps);
         }
         for (int a = 0; a < C::kABufs; ++a) {
-            mbar_init(&afull[a], kDequantThreads / 32);
+            mbar_init(&afull[a], kDequantWarps);
             mbar_init(&aempty[a], 1);
         }
         mbar_init(tfull, 1);
@@ -132,23 +145,30 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
 
-    if (warp == 0) {
+    if (warp == 0 || warp == 2) {
         if (lane == 0) {
-            // ---------------- TMA producer ----------------
+            // ---------------- TMA: X ring (warp 0) or packed-weight ring (warp 2) ----------------
+            const bool xs = warp == 0;
+            const int S = xs ? C::kXStages : C::kWStages;
+            uint64_t* full = xs ? xfull : wfull;
+            uint64_t* empty = xs ? xempty : wempty;
+            const uint32_t bytes = xs ? C::kXBytes : C::kWBytes;
+            uint8_t* base = smem + (xs ? C::kXOff : C::kWOff);
             int issued = 0;
             bool ok = true;
             for (int kb = 0; kb < num_kb && ok; ++kb) {
-                const int s = kb % C::kStages;
-                if (kb >= C::kStages) ok = mbar_wait(&empty[s], ((kb / C::kStages) - 1) & 1);
+                const int s = kb % S;
+                if (kb >= S) ok = mbar_wait(&empty[s], ((kb / S) - 1) & 1);
                 if (!ok) break;
-                mbar_arrive_expect_tx(&full[s], C::kXBytes + C::kWBytes);
-                tma_load_2d(smem + C::kXOff + s * C::kXBytes, &tmap_x, &full[s], (kb0 + kb) * kGemmKB, m0);
-                tma_load_2d(smem + C::kWOff + s * C::kWBytes, &tmap_q, &full[s], (kb0 + kb) * (kGemmKB / 8), n0);
+                mbar_arrive_expect_tx(&full[s], bytes);
+                if (xs)
+                    tma_load_2d(base + s * bytes, &tmap_x, &full[s], (kb0 + kb) * kGemmKB, m0);
+                else
+                    tma_load_2d(base + s * bytes, &tmap_q, &full[s], (kb0 + kb) * (kGemmKB / 8), n0);
                 ++issued;
             }
             // Drain: every issued copy must land before the CTA may exit.
-            for (int kb = issued - 1; kb >= 0 && kb >= issued - C::kStages; --kb)
-                mbar_wait(&full[kb % C::kStages], (kb / C::kStages) & 1);
+            for (int kb = issued - 1; kb >= 0 && kb >= issued - S; --kb) mbar_wait(&full[kb % S], (kb / S) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -156,9 +176,9 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
             constexpr uint32_t idesc = idesc_f16_f32(kGemmTileN, BN);
             bool ok = true;
             for (int kb = 0; kb < num_kb && ok; ++kb) {
-                const int s = kb % C::kStages;
+                const int s = kb % C::kXStages;
                 const int a = kb % C::kABufs;
-                ok = mbar_wait(&full[s], (kb / C::kStages) & 1) && mbar_wait(&afull[a], (kb / C::kABufs) & 1);
+                ok = mbar_wait(&xfull[s], (kb / C::kXStages) & 1) && mbar_wait(&afull[a], (kb / C::kABufs) & 1);
                 if (!ok) break;
                 tc_fence_after();
                 const uint64_t adesc = desc_sw128_kmajor(smem_u32(smem + C::kAOff + a * C::kABytes));
@@ -166,7 +186,7 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
 #pragma unroll
                 for (int kk = 0; kk < kGemmKB / 16; ++kk)
                     mma_f16(tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
-                mma_commit(&empty[s]);
+                mma_commit(&xempty[s]);
                 mma_commit(&aempty[a]);
             }
             mma_commit(tfull);   // also on the error path, so that the MMAs drain before TMEM is freed
@@ -174,7 +194,7 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         }
     } else {
         // ---------------- dequantise, then epilogue ----------------
-        const int d = threadIdx.x - 64;           // 0..511
+        const int d = threadIdx.x - 96;           // 0..511
         const int row = d & (kGemmTileN - 1);
         const int kq = d >> 7;                    // which 16 channels of the k-block
         const int n = n0 + row;
@@ -184,8 +204,8 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         const bool row_ok = n < N;
         const uint16_t* srow = scales + (size_t)(row_ok ? n : 0) * ng;
         const uint32_t* zrow = qzeros + (size_t)(row_ok ? n : 0) * nzw;
-        // scale and zero word of the thread's group, loaded one k-block ahead (raw; using a
-        // loaded value stalls on its load) and only when the group changes
+        // scale and zero word of the thread's next group, fetched a group ahead (raw; using
+        // a loaded value stalls on its load)
         const int g_first = (kb0 * kGemmKB + kq * 16) / G;
         uint32_t sc_next = row_ok ? __ldg(srow + g_first) : 0u;
         uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_first >> 3)) : 0u;
@@ -195,12 +215,17 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         constexpr int D = C::kBatch;
         for (int kb = 0; kb < num_kb && ok; kb += D) {
             // the batch's A buffers free and its packed tiles landed
+            uint2 packed[D];
 #pragma unroll
             for (int i = 0; i < D; ++i) {
                 const int kbi = kb + i;
+                packed[i] = make_uint2(0u, 0u);
                 if (kbi < num_kb) {
                     if (kbi >= C::kABufs) ok = ok && mbar_wait(&aempty[kbi % C::kABufs], ((kbi / C::kABufs) - 1) & 1);
-                    ok = ok && mbar_wait(&full[kbi % C::kStages], (kbi / C::kStages) & 1);
+                    ok = ok && mbar_wait(&wfull[kbi % C::kWStages], (kbi / C::kWStages) & 1);
+                    if (ok)
+                        packed[i] = *reinterpret_cast<const uint2*>(smem + C::kWOff + (kbi % C::kWStages) * C::kWBytes +
+                                                                    row * 32 + kq * 8);
                 }
             }
             if (!ok) break;
@@ -232,27 +257,27 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                         if (zp) zw_next = __ldg(zrow + (gn >> 3));
                     }
                 }
-                const int s = kbi % C::kStages;
-                const uint2 packed =
-                    *reinterpret_cast<const uint2*>(smem + C::kWOff + s * C::kWBytes + row * 32 + kq * 8);
                 uint8_t* atile = smem + C::kAOff + (kbi % C::kABufs) * C::kABytes;
-                const uint4 v0 = live ? dequant_word(packed.x, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
-                const uint4 v1 = live ? dequant_word(packed.y, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+                const uint4 v0 = live ? dequant_word(packed[i].x, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
+                const uint4 v1 = live ? dequant_word(packed[i].y, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4*>(atile + sw128_offset(row, kq * 2)) = v0;
                 *reinterpret_cast<uint4*>(atile + sw128_offset(row, kq * 2 + 1)) = v1;
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
+            if (lane == 0) {   // the packed words have been used: their slots go back to the producer
 #pragma unroll
                 for (int i = 0; i < D; ++i)
-                    if (kb + i < num_kb) mbar_arrive(&afull[(kb + i) % C::kABufs]);
+                    if (kb + i < num_kb) {
+                        mbar_arrive(&wempty[(kb + i) % C::kWStages]);
+                        mbar_arrive(&afull[(kb + i) % C::kABufs]);
+                    }
             }
         }
         if (ok && mbar_wait(tfull, 0)) {
             tc_fence_after();
             const int q = warp & 3;                        // TMEM lane quarter this warp may access
-            const int set = (warp - 2) >> 2;               // 0..3: four warps per lane quarter
+            const int set = (warp - 3) >> 2;               // 0..3: four warps per lane quarter
             const int cols = BN >= 64 ? BN / 4 : 16;
             const int c_begin = set * cols;
             if (c_begin < BN) {
