@@ -13,15 +13,18 @@
 // and each group keeps the ratio with the smallest error (ties to the smaller j: less
 // clipping), then is quantised clipped at it.
 //
-// One CTA takes 128 output channels, 256 calibration tokens and a run of groups.  For a
-// group its producer warps find the group's extremes once; then for each ratio they
-// build dW_j 2^e as fp16 hi + lo tiles (the construction of the fused scale search; the
-// exponent comes from the same bound), one tcgen05.mma chain per (group, ratio) puts
-// E = X_g dW_j^T in one of two 256-column TMEM accumulators, and while the next one
-// fills, the producers drain this one: per row the sum over the tokens of E^2 (fp32 over
-// 16 tokens, fp64 beyond), the four warps of a row combined in a fixed order.  The
-// errors of the CTA's token chunk go to err_part; a second kernel adds the chunks in a
-// fixed order, picks the ratio and packs.
+// One CTA takes 128 output channels, 512 calibration tokens (256 at G = 256) and a run
+// of groups.  For a group its producer warps find the group's extremes once; then for
+// each ratio they build dW_j 2^e as fp16 hi + lo tiles (the construction of the fused
+// scale search; the exponent comes from the same bound), and one tcgen05.mma chain per
+// (group, ratio) puts E = X_g dW_j^T in TMEM: with 512 tokens the same dW tile feeds two
+// 256-column accumulators (one per 256 tokens), with 256 tokens two tiles alternate
+// between them so that one fills while the other drains.  The producers drain a tile
+// after building the next: per row the sum over the tokens of E^2 (fp32 over 16 tokens,
+// fp64 beyond), the four warps of a row combined in a fixed order.  The errors of the
+// CTA's token chunk go to err_part; a second kernel adds the chunks in a fixed order,
+// picks the ratio and packs.
+
 #pragma once
 
 #include "common.cuh"
@@ -33,27 +36,35 @@ namespace awq {
 
 constexpr int kClipMaxRatios = 32;
 constexpr int kClipRows = 128;
-constexpr int kClipTokens = 256;
 constexpr int kClipABufs = 2;
+
+// Tokens per CTA: 512 up to G = 128, so that each dW tile (group, ratio) feeds two
+// 256-column accumulators (half the producer work per multiply-add of 256 tokens); 256 at
+// G = 256, whose X for a group (4 blocks) would not fit twice as long.
+__host__ __device__ constexpr int clip_tokens(int G) { return G >= 256 ? 256 : 512; }
 constexpr int kClipProducerWarps = 16;
 constexpr int kClipThreads = 64 + kClipProducerWarps * 32;
 
 template <int G>
 struct ClipCfg {
+    static constexpr int kTok = clip_tokens(G);
+    static constexpr int kHalves = kTok / 256;                      // 256-column accumulators per tile
+    static constexpr int kAccSets = kHalves == 1 ? 2 : 1;           // tiles held in TMEM (512 columns)
     static constexpr int kSub = G >= 64 ? G / 64 : 1;              // 64-channel blocks per group
-    static constexpr int kXSlots = G >= 256 ? 1 : 2;                // groups of X held
-    static constexpr int kXTileBytes = kClipTokens * 128;           // 256 tokens x 64 channels
+    static constexpr int kXSlots = G >= 128 ? 1 : 2;                // groups of X held
+    static constexpr int kXTileBytes = kTok * 128;                  // kTok tokens x 64 channels
     static constexpr int kXSlotBytes = kSub * kXTileBytes;
     static constexpr int kATileBytes = kClipRows * 128;
     static constexpr int kABufBytes = 2 * kATileBytes;              // hi, lo
     static constexpr int kXOff = 0;
     static constexpr int kAOff = kXSlots * kXSlotBytes;
     static constexpr int kBarOff = kAOff + kClipABufs * kABufBytes;
-    // xfull, xempty [kXSlots]; afull, aempty [kClipABufs]; accfull, accempty [2]; done
-    static constexpr int kNumBars = 2 * kXSlots + 2 * kClipABufs + 5;
+    // xfull, xempty [kXSlots]; afull, aempty [kClipABufs]; accfull, accempty [kAccSets]; done
+    static constexpr int kNumBars = 2 * kXSlots + 2 * kClipABufs + 2 * kAccSets + 1;
     static constexpr int kRedOff = kBarOff + kNumBars * 8;          // [2][128][4] double
     static constexpr int kTmemPtrOff = kRedOff + 2 * kClipRows * 4 * 8;
     static constexpr int kSmemBytes = kTmemPtrOff + 16 + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory of one CTA exceeds 227 KB");
 };
 
 // s as fp32 and the group extremes of s for the exponent bound (one table slot), for a
@@ -86,7 +97,7 @@ __device__ __forceinline__ float clip_ratio(int j, int n_grid) {
     return __double2float_rn(__dsub_rn(1.0, __ddiv_rn((double)j, (double)n_grid)));
 }
 
-// grid = (row blocks of 128, token chunks of 256, runs of groups); err_part
+// grid = (row blocks of 128, token chunks of clip_tokens(G), runs of groups); err_part
 // [token chunk][N][ng][n_clip].
 template <int G>
 __global__ void __launch_bounds__(kClipThreads, 1)
@@ -104,16 +115,16 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
     uint64_t* xempty = xfull + C::kXSlots;
     uint64_t* afull = xempty + C::kXSlots;
     uint64_t* aempty = afull + kClipABufs;
-    uint64_t* accfull = aempty + kClipABufs;     // [2]
-    uint64_t* accempty = accfull + 2;            // [2]
-    uint64_t* done = accempty + 2;               // every MMA of the CTA complete
+    uint64_t* accfull = aempty + kClipABufs;     // [kAccSets]
+    uint64_t* accempty = accfull + C::kAccSets;  // [kAccSets]
+    uint64_t* done = accempty + C::kAccSets;     // every MMA of the CTA complete
     double* red = reinterpret_cast<double*>(smem + C::kRedOff);
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::kTmemPtrOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kClipRows;
     const int tc = blockIdx.y;
-    const int m0 = tc * kClipTokens;
+    const int m0 = tc * C::kTok;
     const int ng = K / G;
     const int g_begin = blockIdx.z * groups_per_cta;
     const int g_end = min(ng, g_begin + groups_per_cta);
@@ -129,7 +140,7 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
             mbar_init(&afull[b], kClipProducerWarps);
             mbar_init(&aempty[b], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::kAccSets; ++b) {
             mbar_init(&accfull[b], 1);
             mbar_init(&accempty[b], kClipProducerWarps);
         }
@@ -158,8 +169,9 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
                 const int kbase = ((g_begin + gi) * G) & ~63;
                 mbar_arrive_expect_tx(&xfull[slot], (uint32_t)(U * C::kXTileBytes));
                 for (int u = 0; u < U; ++u)
-                    tma_load_2d(smem + C::kXOff + slot * C::kXSlotBytes + u * C::kXTileBytes, &tmap_x, &xfull[slot],
-                                kbase + u * 64, m0);
+                    for (int h = 0; h < C::kHalves; ++h)   // boxes of 256 tokens
+                        tma_load_2d(smem + C::kXOff + slot * C::kXSlotBytes + u * C::kXTileBytes + h * 256 * 128,
+                                    &tmap_x, &xfull[slot], kbase + u * 64, m0 + h * 256);
                 ++issued;
             }
             for (int gi = issued - 1; gi >= 0 && gi >= issued - C::kXSlots; --gi)
@@ -168,17 +180,17 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA: one accumulator chain per (group, ratio) ----------------
-            constexpr uint32_t idesc = idesc_f16_f32(kClipRows, kClipTokens);
+            constexpr uint32_t idesc = idesc_f16_f32(kClipRows, 256);
             bool ok = true;
             int sub = 0;                                   // A sub-tiles consumed
             for (int t = 0; t < n_tiles && ok; ++t) {
                 const int gi = t / n_clip, j = t - gi * n_clip;
                 const int slot = gi % C::kXSlots;
-                const int acc = t & 1;
+                const int acc = t % C::kAccSets;
                 if (j == 0) ok = mbar_wait(&xfull[slot], (gi / C::kXSlots) & 1);
-                if (ok && t >= 2) ok = mbar_wait(&accempty[acc], ((t >> 1) - 1) & 1);
+                if (ok && t >= C::kAccSets) ok = mbar_wait(&accempty[acc], ((t / C::kAccSets) - 1) & 1);
                 if (!ok) break;
-                const uint32_t d = tmem + (uint32_t)(acc * kClipTokens);
+                const uint32_t d = tmem + (uint32_t)(acc * C::kHalves * 256);
                 const int kk0 = G >= 64 ? 0 : (((g_begin + gi) & 1) * 2);    // G = 32: the half of the block
                 for (int u = 0; u < U && ok; ++u, ++sub) {
                     const int b = sub % kClipABufs;
@@ -187,13 +199,17 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
                     tc_fence_after();
                     const uint32_t abase = smem_u32(smem + C::kAOff + b * C::kABufBytes);
                     const uint64_t ah = desc_sw128_kmajor(abase), al = desc_sw128_kmajor(abase + C::kATileBytes);
-                    const uint64_t bd =
-                        desc_sw128_kmajor(smem_u32(smem + C::kXOff + slot * C::kXSlotBytes + u * C::kXTileBytes));
+                    const uint32_t xb = smem_u32(smem + C::kXOff + slot * C::kXSlotBytes + u * C::kXTileBytes);
 #pragma unroll
                     for (int kq = 0; kq < kKSteps; ++kq) {
                         const int kk = kk0 + kq;
-                        mma_f16(d, ah + 2 * kk, bd + 2 * kk, idesc, (u | kq) != 0);
-                        mma_f16(d, al + 2 * kk, bd + 2 * kk, idesc, 1u);
+#pragma unroll
+                        for (int h = 0; h < C::kHalves; ++h) {   // the same dW feeds every 256 tokens
+                            const uint64_t bd = desc_sw128_kmajor(xb + h * 256 * 128);
+                            const uint32_t dh = d + (uint32_t)(h * 256);
+                            mma_f16(dh, ah + 2 * kk, bd + 2 * kk, idesc, (u | kq) != 0);
+                            mma_f16(dh, al + 2 * kk, bd + 2 * kk, idesc, 1u);
+                        }
                     }
                     mma_commit(&aempty[b]);
                 }
@@ -221,17 +237,19 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
         bool ok = true;
         int sub = 0;
 
-        // drain tile t: rows q4*32 + lane, this warp's 64 of the 256 token columns
+        // drain tile t: rows q4*32 + lane, this warp's quarter of the tile's token columns
         auto drain = [&](int t) {
-            const int acc = t & 1;
+            constexpr int kCols = C::kTok / 4;
+            const int acc = t % C::kAccSets;
             double part = 0.0;
-            if (ok) ok = mbar_wait(&accfull[acc], (t >> 1) & 1);
+            if (ok) ok = mbar_wait(&accfull[acc], (t / C::kAccSets) & 1);
             if (ok) {
                 tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < 64; c += 16) {
+#pragma unroll 2
+                for (int c = 0; c < kCols; c += 16) {
                     uint32_t v[16];
-                    tmem_ld16(tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kClipTokens + set * 64 + c), v);
+                    tmem_ld16(tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * C::kHalves * 256 + set * kCols + c),
+                              v);
                     tmem_ld_wait();
                     float f = 0.0f;
 #pragma unroll
@@ -505,7 +523,7 @@ inline ClipWorkspace clip_layout(void* base, int M, int N, int K, int G, int n_c
     w.s32 = reinterpret_cast<float*>(take((size_t)K * 4));
     w.rse = reinterpret_cast<float*>(take((size_t)K * 4));
     w.eexp = reinterpret_cast<int32_t*>(take(4));
-    w.err = reinterpret_cast<double*>(take((size_t)ceil_div(M, kClipTokens) * N * ng * n_clip * 8));
+    w.err = reinterpret_cast<double*>(take((size_t)ceil_div(M, clip_tokens(G)) * N * ng * n_clip * 8));
     w.bytes = off;
     return w;
 }
@@ -545,17 +563,22 @@ inline awq_status run_apply_clip(const uint16_t* X, int M, const uint16_t* W, co
     search_rse_kernel<<<dim3(ceil_div(K, 256), 1), 256, 0, st>>>(w.s32, w.bound, K, 0, w.rse, w.eexp);
     if (cudaGetLastError() != cudaSuccess) return AWQ_ERR_CUDA;
     CUtensorMap tx;
-    if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)M, (uint64_t)K, kClipTokens, 64,
+    if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)M, (uint64_t)K, 256, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B))
         return AWQ_ERR_CUDA;
     const void* fn = clip_err_fn(G);
     if (!prepare_kernel(fn)) return AWQ_ERR_CUDA;
-    // split the groups so that the grid covers the GPU about twice
-    const int rb = ceil_div(N, kClipRows), tcs = ceil_div(M, kClipTokens);
-    int splits = ceil_div(2 * sms, rb * tcs);
-    splits = max(1, min(splits, ng));
-    const int gpc = ceil_div(ng, splits);
-    splits = ceil_div(ng, gpc);
+    // runs of groups per CTA: the count that minimises waves x (groups per CTA + a start-up
+    // of about a third of a group's work)
+    const int rb = ceil_div(N, kClipRows), tcs = ceil_div(M, clip_tokens(G));
+    int gpc = ng;
+    double best = 1e300;
+    for (int c = 1; c <= ng; ++c) {
+        const long long ctas = (long long)rb * tcs * ceil_div(ng, c);
+        const double t = (double)((ctas + sms - 1) / sms) * (c + 0.3);
+        if (t < best * 0.999) best = t, gpc = c;
+    }
+    const int splits = ceil_div(ng, gpc);
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(rb, tcs, splits);
     lc.blockDim = dim3(kClipThreads);
