@@ -97,12 +97,14 @@ __device__ __forceinline__ float clip_ratio(int j, int n_grid) {
     return __double2float_rn(__dsub_rn(1.0, __ddiv_rn((double)j, (double)n_grid)));
 }
 
-// grid = (row blocks of 128, token chunks of clip_tokens(G), runs of groups); err_part
-// [token chunk][N][ng][n_clip].
+// grid = (CTAs sharing the units, token chunks of clip_tokens(G)).  A unit is (block of
+// 128 output channels, group), in the order block-major; CTA c takes the units
+// [c U / P, (c + 1) U / P) of the U = ceil(N / 128) ng, so that the CTAs of a wave get
+// equal work whatever the block and group counts.  err_part [token chunk][N][ng][n_clip].
 template <int G>
 __global__ void __launch_bounds__(kClipThreads, 1)
 clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ W, int M, int N, int K,
-                int zero_point, int n_grid, int n_clip, int groups_per_cta, const float* __restrict__ s32,
+                int zero_point, int n_grid, int n_clip, int n_units, const float* __restrict__ s32,
                 const float* __restrict__ rse, const int32_t* __restrict__ eexp, double* __restrict__ err_part) {
     using C = ClipCfg<G>;
     using namespace sm100;
@@ -122,14 +124,16 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::kTmemPtrOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * kClipRows;
+    const int u_begin = (int)((long long)blockIdx.x * n_units / gridDim.x);
+    const int u_end = (int)((long long)(blockIdx.x + 1) * n_units / gridDim.x);
     const int tc = blockIdx.y;
     const int m0 = tc * C::kTok;
     const int ng = K / G;
-    const int g_begin = blockIdx.z * groups_per_cta;
-    const int g_end = min(ng, g_begin + groups_per_cta);
-    const int n_groups = max(0, g_end - g_begin);
+    const int n_groups = u_end - u_begin;                // units of this CTA
     const int n_tiles = n_groups * n_clip;
+    // group and first output channel of the CTA's unit gi
+    auto unit_g = [&](int gi) { return (u_begin + gi) % ng; };
+    auto unit_n0 = [&](int gi) { return ((u_begin + gi) / ng) * kClipRows; };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kXSlots; ++i) {
@@ -166,7 +170,7 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
                 const int slot = gi % C::kXSlots;
                 if (gi >= C::kXSlots) ok = mbar_wait(&xempty[slot], ((gi / C::kXSlots) - 1) & 1);
                 if (!ok) break;
-                const int kbase = ((g_begin + gi) * G) & ~63;
+                const int kbase = (unit_g(gi) * G) & ~63;
                 mbar_arrive_expect_tx(&xfull[slot], (uint32_t)(U * C::kXTileBytes));
                 for (int u = 0; u < U; ++u)
                     for (int h = 0; h < C::kHalves; ++h)   // boxes of 256 tokens
@@ -191,7 +195,7 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
                 if (ok && t >= C::kAccSets) ok = mbar_wait(&accempty[acc], ((t / C::kAccSets) - 1) & 1);
                 if (!ok) break;
                 const uint32_t d = tmem + (uint32_t)(acc * C::kHalves * 256);
-                const int kk0 = G >= 64 ? 0 : (((g_begin + gi) & 1) * 2);    // G = 32: the half of the block
+                const int kk0 = G >= 64 ? 0 : ((unit_g(gi) & 1) * 2);        // G = 32: the half of the block
                 for (int u = 0; u < U && ok; ++u, ++sub) {
                     const int b = sub % kClipABufs;
                     ok = mbar_wait(&afull[b], (sub / kClipABufs) & 1);
@@ -228,10 +232,7 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
         const int r = dt >> 2;                         // channel row of the tile
         const int qq = dt & 3;                         // quarter of the group's channels in a block
         constexpr int CPT = G >= 64 ? 16 : 8;          // channels of a block per thread
-        const int n = n0 + r;
-        const bool row_ok = n < N;
         const bool zp = zero_point != 0;
-        const uint16_t* wrow = W + (size_t)(row_ok ? n : 0) * K;
         const double undo = ldexp(1.0, -eexp[0]);
         const int q4 = warp & 3, set = pw >> 2;
         bool ok = true;
@@ -271,17 +272,20 @@ clip_err_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __re
             asm volatile("bar.sync %0, %1;" ::"r"(2 + q4), "n"(4 * 32) : "memory");
             if (set == 0) {
                 const int rr = q4 * 32 + lane;
-                const int nn = n0 + rr;
                 const int gi = t / n_clip, j = t - gi * n_clip;
+                const int nn = unit_n0(gi) + rr;
                 const double* q = rb + rr * 4;
                 const double sum = ((q[0] + q[1]) + q[2]) + q[3];
                 if (nn < N)
-                    err_part[(((size_t)tc * N + nn) * ng + (g_begin + gi)) * n_clip + j] = sum * undo * undo;
+                    err_part[(((size_t)tc * N + nn) * ng + unit_g(gi)) * n_clip + j] = sum * undo * undo;
             }
         };
 
         for (int gi = 0; gi < n_groups; ++gi) {
-            const int g = g_begin + gi;
+            const int g = unit_g(gi);
+            const int n = unit_n0(gi) + r;                 // this thread's output channel
+            const bool row_ok = n < N;
+            const uint16_t* wrow = W + (size_t)(row_ok ? n : 0) * K;
             // pass 1: the group's weights (kept packed), ws extremes
             uint32_t wpk[U][CPT / 2];
             float mx = -INFINITY, mn = INFINITY;
@@ -568,19 +572,13 @@ inline awq_status run_apply_clip(const uint16_t* X, int M, const uint16_t* W, co
         return AWQ_ERR_CUDA;
     const void* fn = clip_err_fn(G);
     if (!prepare_kernel(fn)) return AWQ_ERR_CUDA;
-    // runs of groups per CTA: the count that minimises waves x (groups per CTA + a start-up
-    // of about a third of a group's work)
+    // the (128-channel block, group) units shared evenly by one wave of CTAs (or all units
+    // when there are fewer)
     const int rb = ceil_div(N, kClipRows), tcs = ceil_div(M, clip_tokens(G));
-    int gpc = ng;
-    double best = 1e300;
-    for (int c = 1; c <= ng; ++c) {
-        const long long ctas = (long long)rb * tcs * ceil_div(ng, c);
-        const double t = (double)((ctas + sms - 1) / sms) * (c + 0.3);
-        if (t < best * 0.999) best = t, gpc = c;
-    }
-    const int splits = ceil_div(ng, gpc);
+    const int n_units = rb * ng;
+    const int ctas = max(1, min(n_units, max(1, sms / tcs)));
     cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3(rb, tcs, splits);
+    lc.gridDim = dim3(ctas, tcs);
     lc.blockDim = dim3(kClipThreads);
     lc.dynamicSmemBytes = clip_smem_bytes(G);
     lc.stream = st;
@@ -588,8 +586,8 @@ inline awq_status run_apply_clip(const uint16_t* X, int M, const uint16_t* W, co
     const float* rse = w.rse;
     const int32_t* eexp = w.eexp;
     double* err = w.err;
-    int gpc_arg = gpc;
-    void* args[] = {&tx, &W, &M, &N, &K, &zp, &n_grid, &n_clip, &gpc_arg, &s32, &rse, &eexp, &err};
+    int units_arg = n_units;
+    void* args[] = {&tx, &W, &M, &N, &K, &zp, &n_grid, &n_clip, &units_arg, &s32, &rse, &eexp, &err};
     if (cudaLaunchKernelExC(&lc, fn, args) != cudaSuccess) return AWQ_ERR_CUDA;
     const long long blocks = (long long)ceil_div(N, kQuantRows) * ceil_div(K, kQuantChunk);
     clip_pack_kernel<<<(unsigned)blocks, kQuantThreads, 0, st>>>(W, s, N, K, G, zp, n_grid, n_clip, tcs, w.err,
