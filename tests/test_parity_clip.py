@@ -48,7 +48,7 @@ def _check(lib, X, W, s, G, zp, n_grid=20, n_clip=10):
     return idx, worst
 
 
-SHAPES = [(64, 256, 128), (300, 512, 200), (40, 1024, 130), (512, 256, 64)]
+SHAPES = [(64, 256, 128), (300, 512, 200), (40, 1024, 130), (512, 256, 64), (700, 512, 200)]
 
 
 @pytest.mark.parametrize("G", O.GROUP_SIZES)
@@ -85,6 +85,17 @@ def test_apply_clip_without_scale_and_grid_variants(lib):
     W[5] = 0
     for n_grid, n_clip in ((20, 10), (10, 4), (32, 32)):
         _check(lib, X, W, None, 32, True, n_grid, n_clip)
+
+
+def test_apply_clip_units_cross_channel_blocks(lib):
+    """More (128-channel block, group) units than one wave of CTAs holds (1300 channels in
+    11 blocks, the last ragged, x 16 groups = 176 units): CTAs take one or two units, some
+    crossing from one block to the next; every error and index against the oracle."""
+    M, K, N, G = 64, 1024, 1300, 64
+    X = inputs.activations(M, K, seed=607)
+    W = inputs.weights(N, K, 0.02, seed=608)
+    s = O.scales_for_alpha(O.act_absmean(X), 0.4)
+    _check(lib, X, W, s, G, True)
 
 
 def test_apply_clip_layer_4096(lib):
