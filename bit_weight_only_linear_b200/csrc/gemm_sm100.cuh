@@ -15,9 +15,10 @@
 //   warp 0      TMA producer of X: tile [BN x 64] fp16 (128B swizzle) per 64-channel k-block,
 //               into a ring whose slots the MMAs free.
 //   warp 1      allocates TMEM; one lane issues 4 tcgen05.mma (K = 16 each) per k-block.
-//   warp 2      TMA producer of the packed weights: tile [128 x 8 words] per k-block, into a
-//               ring of its own whose slots the dequantisers free as soon as they have read
-//               the words, so that refilling it never waits for the MMAs.
+//   warp 2      TMA producer of the packed weights: tile [128 rows x 32 words] = 4 k-blocks per
+//               stage (whole 128-byte lines per row; 32-byte rows cap the copy rate), 128B-
+//               swizzled, into a ring of its own whose slots the dequantisers free as soon
+//               as they have read the words, so that refilling it never waits for the MMAs.
 //   warps 3..18 dequantise: thread (row, quarter) turns 16 codes per k-block into fp16
 //               (q - z) * scale16 with mask/magic-number arithmetic, a batch of k-blocks per
 //               iteration, and writes them in the 128B-swizzled K-major layout the MMA
@@ -41,18 +42,29 @@ constexpr int kGemmTileN = 128;      // output channels per CTA (MMA M)
 constexpr int kGemmKB = 64;          // input channels per k-block
 constexpr int kDequantThreads = kDequantWarps * 32;   // 4 threads per row, 16 codes each
 
+// Byte offset `a` inside a packed-weight stage whose rows are 32 * WKB bytes, as TMA lays it
+// out with the 32 * WKB-byte swizzle (none for one k-block): the 16-byte unit index is
+// XOR-ed with the 128-byte line index, modulo the swizzle span.  The stage starts on a
+// 1024-byte boundary.
+template <int WKB>
+__device__ __forceinline__ uint32_t wstage_swizzle(uint32_t a) {
+    if constexpr (WKB == 1) return a;
+    else return a ^ (((a >> 7) & (uint32_t)(2 * WKB - 1)) << 4);
+}
+
 template <int BN>
 struct GemmCfg {
-    static constexpr int kXStages = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
-    // packed weights: deep enough to keep a DRAM round trip in flight
-    static constexpr int kWStages = BN >= 256 ? 4 : (BN >= 128 ? 8 : (BN >= 64 ? 12 : 16));
-    static constexpr int kABufs = BN >= 256 ? 3 : (BN >= 128 ? 4 : (BN >= 64 ? 6 : 8));
+    static constexpr int kXStages = BN >= 256 ? 4 : (BN >= 64 ? 6 : 8);
+    // packed weights: kWKB k-blocks per stage (rows of one 128-byte line)
+    static constexpr int kWKB = 4;
+    static constexpr int kWStages = BN >= 256 ? 2 : (BN >= 64 ? 3 : 4);
+    static constexpr int kABufs = BN >= 256 ? 3 : (BN >= 128 ? 4 : 8);
     // k-blocks a dequantising thread converts per iteration (one fence and one wait per
     // barrier round trip for all of them); half the A buffers, so that the MMA consumes
     // one batch while the next is written
     static constexpr int kBatch = BN >= 256 ? 1 : kABufs / 2;
     static constexpr int kXBytes = BN * 128;                 // X tile: BN rows x 128 B
-    static constexpr int kWBytes = kGemmTileN * 32;          // packed tile: 128 rows x 32 B
+    static constexpr int kWBytes = kGemmTileN * 32 * kWKB;   // packed stage: 128 rows x 128 B
     static constexpr int kABytes = kGemmTileN * 128;         // dequantised tile
     static constexpr int kXOff = 0;
     static constexpr int kAOff = kXOff + kXStages * kXBytes;  // both multiples of 1024
@@ -63,7 +75,9 @@ struct GemmCfg {
     static constexpr int kSmemBytes = kTmemPtrOff + 16 + 1024;   // + slack to align the base to 1024
     static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
     static_assert(kSmemBytes <= 232448, "shared memory of one CTA exceeds 227 KB");
-    static_assert(kWStages >= kBatch && kXStages >= kBatch && kABufs >= 2 * kBatch || kBatch == 1, "ring depths");
+    static_assert(kXStages >= kBatch && kABufs >= 2 * kBatch || kBatch == 1, "ring depths");
+    static_assert(kWKB % kBatch == 0, "a batch of k-blocks lies in one packed-weight stage");
+    static_assert(kWKB == 4 && kWOff % 1024 == 0, "128-byte swizzled packed stages on 1024-byte boundaries");
 };
 
 // (q - z) * s for the 8 codes of one word, returned as 4 fp16 pairs in k order.  The
@@ -150,25 +164,26 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
             // ---------------- TMA: X ring (warp 0) or packed-weight ring (warp 2) ----------------
             const bool xs = warp == 0;
             const int S = xs ? C::kXStages : C::kWStages;
+            const int n_st = xs ? num_kb : ceil_div(num_kb, C::kWKB);   // one or kWKB k-blocks a stage
             uint64_t* full = xs ? xfull : wfull;
             uint64_t* empty = xs ? xempty : wempty;
             const uint32_t bytes = xs ? C::kXBytes : C::kWBytes;
             uint8_t* base = smem + (xs ? C::kXOff : C::kWOff);
             int issued = 0;
             bool ok = true;
-            for (int kb = 0; kb < num_kb && ok; ++kb) {
-                const int s = kb % S;
-                if (kb >= S) ok = mbar_wait(&empty[s], ((kb / S) - 1) & 1);
+            for (int j = 0; j < n_st && ok; ++j) {
+                const int s = j % S;
+                if (j >= S) ok = mbar_wait(&empty[s], ((j / S) - 1) & 1);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 if (xs)
-                    tma_load_2d(base + s * bytes, &tmap_x, &full[s], (kb0 + kb) * kGemmKB, m0);
+                    tma_load_2d(base + s * bytes, &tmap_x, &full[s], (kb0 + j) * kGemmKB, m0);
                 else
-                    tma_load_2d(base + s * bytes, &tmap_q, &full[s], (kb0 + kb) * (kGemmKB / 8), n0);
+                    tma_load_2d(base + s * bytes, &tmap_q, &full[s], (kb0 + j * C::kWKB) * (kGemmKB / 8), n0);
                 ++issued;
             }
             // Drain: every issued copy must land before the CTA may exit.
-            for (int kb = issued - 1; kb >= 0 && kb >= issued - S; --kb) mbar_wait(&full[kb % S], (kb / S) & 1);
+            for (int j = issued - 1; j >= 0 && j >= issued - S; --j) mbar_wait(&full[j % S], (j / S) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -202,11 +217,12 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         const int nzw = ceil_div(ng, 8);
         const bool zp = zero_point != 0;
         const bool row_ok = n < N;
+        const int lg = 31 - __clz(G);             // G is a power of two
         const uint16_t* srow = scales + (size_t)(row_ok ? n : 0) * ng;
         const uint32_t* zrow = qzeros + (size_t)(row_ok ? n : 0) * nzw;
         // scale and zero word of the thread's next group, fetched a group ahead (raw; using
         // a loaded value stalls on its load)
-        const int g_first = (kb0 * kGemmKB + kq * 16) / G;
+        const int g_first = (kb0 * kGemmKB + kq * 16) >> lg;
         uint32_t sc_next = row_ok ? __ldg(srow + g_first) : 0u;
         uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_first >> 3)) : 0u;
         int g_cur = -1;
@@ -222,10 +238,12 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                 packed[i] = make_uint2(0u, 0u);
                 if (kbi < num_kb) {
                     if (kbi >= C::kABufs) ok = ok && mbar_wait(&aempty[kbi % C::kABufs], ((kbi / C::kABufs) - 1) & 1);
-                    ok = ok && mbar_wait(&wfull[kbi % C::kWStages], (kbi / C::kWStages) & 1);
+                    const int j = kbi / C::kWKB, sb = kbi % C::kWKB;   // stage, k-block inside it
+                    if (i == 0) ok = ok && mbar_wait(&wfull[j % C::kWStages], (j / C::kWStages) & 1);
                     if (ok)
-                        packed[i] = *reinterpret_cast<const uint2*>(smem + C::kWOff + (kbi % C::kWStages) * C::kWBytes +
-                                                                    row * 32 + kq * 8);
+                        packed[i] = *reinterpret_cast<const uint2*>(
+                            smem + C::kWOff + (j % C::kWStages) * C::kWBytes +
+                            wstage_swizzle<C::kWKB>(row * (32 * C::kWKB) + sb * 32 + kq * 8));
                 }
             }
             if (!ok) break;
@@ -235,7 +253,7 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                 if (kbi >= num_kb) break;
                 const int k = (kb0 + kbi) * kGemmKB + kq * 16;
                 const bool live = row_ok && k < K;
-                const int g_here = k / G;
+                const int g_here = k >> lg;
                 if (live && g_here != g_cur) {   // sc_next / zw_next hold this group's parameters
                     g_cur = g_here;
                     const uint32_t sc = sc_next;
@@ -251,8 +269,8 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                     if (!(h2f((uint16_t)sc) * qz_max < 65520.0f) && !isnan(h2f((uint16_t)sc))) raise_error(kErrRange);
                     // the next group this thread reaches (G / 64 k-blocks on, at least one): its
                     // parameters are fetched now, a whole group ahead of their use
-                    const int gn = g_cur + (G >= kGemmKB ? 1 : kGemmKB / G);
-                    if (gn * G < K) {
+                    const int gn = g_cur + (lg >= 6 ? 1 : (kGemmKB >> lg));
+                    if ((gn << lg) < K) {
                         sc_next = __ldg(srow + gn);
                         if (zp) zw_next = __ldg(zrow + (gn >> 3));
                     }
@@ -265,13 +283,16 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {   // the packed words have been used: their slots go back to the producer
+            if (lane == 0) {   // the packed words have been used: a finished stage goes back to the producer
 #pragma unroll
-                for (int i = 0; i < D; ++i)
-                    if (kb + i < num_kb) {
-                        mbar_arrive(&wempty[(kb + i) % C::kWStages]);
-                        mbar_arrive(&afull[(kb + i) % C::kABufs]);
+                for (int i = 0; i < D; ++i) {
+                    const int kbi = kb + i;
+                    if (kbi < num_kb) {
+                        if (kbi % C::kWKB == C::kWKB - 1 || kbi == num_kb - 1)
+                            mbar_arrive(&wempty[(kbi / C::kWKB) % C::kWStages]);
+                        mbar_arrive(&afull[kbi % C::kABufs]);
                     }
+                }
             }
         }
         if (ok && mbar_wait(tfull, 0)) {
@@ -318,7 +339,7 @@ gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
 // ring (freed by the MMAs) is the only round trip on the MMA's critical path.
 //   warp 0     TMA: X tiles [256 tokens x 64] into the X ring
 //   warp 1     TMEM allocation; one lane issues 8 tcgen05.mma per k-block
-//   warp 2     TMA: packed tiles [256 rows x 8 words] into the W ring
+//   warp 2     TMA: packed tiles [256 rows x 8 kWKB words] (kWKB k-blocks) into the W ring
 //   warps 3-18 dequantise (thread = row, 32 codes), then the epilogue
 // ---------------------------------------------------------------------------
 constexpr int kWideRows = 256;
@@ -326,11 +347,13 @@ constexpr int kWideBN = 256;
 constexpr int kWideThreads = 96 + kDequantWarps * 32;
 
 struct GemmWideCfg {
-    static constexpr int kXStages = 4;
-    static constexpr int kWStages = 4;
+    // packed weights: kWKB k-blocks per stage, rows of 32 kWKB bytes (swizzled to match)
+    static constexpr int kWKB = 1;
+    static constexpr int kXStages = kWKB >= 4 ? 3 : 4;
+    static constexpr int kWStages = kWKB >= 2 ? 2 : 4;
     static constexpr int kABufs = 2;
     static constexpr int kXBytes = kWideBN * 128;              // 256 tokens x 64 fp16
-    static constexpr int kWBytes = kWideRows * 32;             // 256 rows x 8 words
+    static constexpr int kWBytes = kWideRows * 32 * kWKB;      // 256 rows x 8 kWKB words
     static constexpr int kATileBytes = kGemmTileN * 128;       // one 128-channel tile
     static constexpr int kABytes = 2 * kATileBytes;
     static constexpr int kXOff = 0;
@@ -340,6 +363,8 @@ struct GemmWideCfg {
     static constexpr int kNumBars = 2 * kXStages + 2 * kWStages + 2 * kABufs + 1;
     static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kTmemPtrOff + 16 + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory of one CTA exceeds 227 KB");
+    static_assert((kWKB == 1 || kWKB == 2 || kWKB == 4) && kWOff % 1024 == 0, "swizzled packed stages");
 };
 
 __global__ void __launch_bounds__(kWideThreads, 1)
@@ -398,24 +423,25 @@ gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
             // ---------------- TMA: X ring (warp 0) or packed-weight ring (warp 2) ----------------
             const bool xs = warp == 0;
             const int S = xs ? C::kXStages : C::kWStages;
+            const int n_st = xs ? num_kb : ceil_div(num_kb, C::kWKB);   // one or kWKB k-blocks a stage
             uint64_t* full = xs ? xfull : wfull;
             uint64_t* empty = xs ? xempty : wempty;
             const uint32_t bytes = xs ? C::kXBytes : C::kWBytes;
             uint8_t* base = smem + (xs ? C::kXOff : C::kWOff);
             int issued = 0;
             bool ok = true;
-            for (int kb = 0; kb < num_kb && ok; ++kb) {
-                const int s = kb % S;
-                if (kb >= S) ok = mbar_wait(&empty[s], ((kb / S) - 1) & 1);
+            for (int j = 0; j < n_st && ok; ++j) {
+                const int s = j % S;
+                if (j >= S) ok = mbar_wait(&empty[s], ((j / S) - 1) & 1);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 if (xs)
-                    tma_load_2d(base + s * bytes, &tmap_x, &full[s], kb * kGemmKB, m0);
+                    tma_load_2d(base + s * bytes, &tmap_x, &full[s], j * kGemmKB, m0);
                 else
-                    tma_load_2d(base + s * bytes, &tmap_q, &full[s], kb * (kGemmKB / 8), n0);
+                    tma_load_2d(base + s * bytes, &tmap_q, &full[s], j * C::kWKB * (kGemmKB / 8), n0);
                 ++issued;
             }
-            for (int kb = issued - 1; kb >= 0 && kb >= issued - S; --kb) mbar_wait(&full[kb % S], (kb / S) & 1);
+            for (int j = issued - 1; j >= 0 && j >= issued - S; --j) mbar_wait(&full[j % S], (j / S) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -453,20 +479,22 @@ gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
         const int nzw = ceil_div(ng, 8);
         const bool zp = zero_point != 0;
         const bool row_ok = n < N;
+        const int lg = 31 - __clz(G);             // G is a power of two
         const uint16_t* srow = scales + (size_t)(row_ok ? n : 0) * ng;
         const uint32_t* zrow = qzeros + (size_t)(row_ok ? n : 0) * nzw;
-        const int g_first = (kh * 32) / G;
+        const int g_first = (kh * 32) >> lg;
         uint32_t sc_next = row_ok ? __ldg(srow + g_first) : 0u;
         uint32_t zw_next = (row_ok && zp) ? __ldg(zrow + (g_first >> 3)) : 0u;
         int g_cur = -1;
         uint32_t s2 = 0, zmagic = 0x64006400u, zneg16 = 0;
         bool ok = true;
         for (int kb = 0; kb < num_kb && ok; ++kb) {
-            const int s = kb % C::kWStages;
+            const int j = kb / C::kWKB, sb = kb % C::kWKB;   // packed-weight stage, k-block inside it
+            const int s = j % C::kWStages;
             const int a = kb % C::kABufs;
             const int k = kb * kGemmKB + kh * 32;
             const bool live = row_ok && k < K;
-            const int g_here = k / G;
+            const int g_here = k >> lg;
             if (live && g_here != g_cur) {   // sc_next / zw_next hold this group's parameters
                 g_cur = g_here;
                 const uint32_t sc = sc_next;
@@ -480,23 +508,25 @@ gemm_w4a16_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
                 if (!(h2f((uint16_t)sc) * qz_max < 65520.0f) && !isnan(h2f((uint16_t)sc))) raise_error(kErrRange);
                 // the next group this thread reaches (G / 64 k-blocks on, at least one): its
                 // parameters are fetched now, a whole group ahead of their use
-                const int gn = g_cur + (G >= kGemmKB ? 1 : kGemmKB / G);
-                if (gn * G < K) {
+                const int gn = g_cur + (lg >= 6 ? 1 : (kGemmKB >> lg));
+                if ((gn << lg) < K) {
                     sc_next = __ldg(srow + gn);
                     if (zp) zw_next = __ldg(zrow + (gn >> 3));
                 }
             }
-            ok = mbar_wait(&wfull[s], (kb / C::kWStages) & 1);
+            ok = mbar_wait(&wfull[s], (j / C::kWStages) & 1);
             if (ok && kb >= C::kABufs) ok = mbar_wait(&aempty[a], ((kb / C::kABufs) - 1) & 1);
             if (!ok) break;
-            const uint4 packed = *reinterpret_cast<const uint4*>(smem + C::kWOff + s * C::kWBytes + row * 32 + kh * 16);
+            const uint4 packed = *reinterpret_cast<const uint4*>(
+                smem + C::kWOff + s * C::kWBytes + wstage_swizzle<C::kWKB>(row * (32 * C::kWKB) + sb * 32 + kh * 16));
             uint4 v[4];
             v[0] = live ? dequant_word(packed.x, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
             v[1] = live ? dequant_word(packed.y, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
             v[2] = live ? dequant_word(packed.z, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
             v[3] = live ? dequant_word(packed.w, zmagic, zneg16, s2) : make_uint4(0, 0, 0, 0);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&wempty[s]);     // the packed words are in registers
+            if (lane == 0 && (sb == C::kWKB - 1 || kb == num_kb - 1))
+                mbar_arrive(&wempty[s]);                // the stage's packed words are in registers
             uint8_t* atile = smem + C::kAOff + a * C::kABytes + rt * C::kATileBytes;
 #pragma unroll
             for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(atile + sw128_offset(r, kh * 4 + c)) = v[c];
@@ -602,14 +632,15 @@ awq_status launch_gemm_bn(const uint16_t* X, int M, const uint32_t* qweight, con
                       CU_TENSOR_MAP_SWIZZLE_128B))
         return AWQ_ERR_CUDA;
     if (!make_tmap_2d(&tq, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)N, (uint64_t)(K / 8), kGemmTileN,
-                      kGemmKB / 8, CU_TENSOR_MAP_SWIZZLE_NONE))
+                      C::kWKB * kGemmKB / 8, CU_TENSOR_MAP_SWIZZLE_128B))
         return AWQ_ERR_CUDA;
     auto kern = gemm_w4a16_kernel<BN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return AWQ_ERR_CUDA;
     const int num_kb = ceil_div(K, kGemmKB);
     if (splits < 1 || part == nullptr) splits = 1;
-    const int kb_per = ceil_div(num_kb, splits);
+    // each split a whole number of packed-weight stages
+    const int kb_per = ceil_div(ceil_div(num_kb, splits), C::kWKB) * C::kWKB;
     splits = ceil_div(num_kb, kb_per);
     dim3 grid(ceil_div(M, BN), ceil_div(N, kGemmTileN), splits);
     if (grid.y > 65535u) return AWQ_ERR_UNSUPPORTED;
@@ -657,8 +688,11 @@ inline awq_status launch_gemm_wide(const uint16_t* X, int M, const uint32_t* qwe
     if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)M, (uint64_t)K, kWideBN, kGemmKB,
                       CU_TENSOR_MAP_SWIZZLE_128B))
         return AWQ_ERR_CUDA;
+    constexpr CUtensorMapSwizzle wswz = C::kWKB == 4   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                        : C::kWKB == 2 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                       : CU_TENSOR_MAP_SWIZZLE_NONE;
     if (!make_tmap_2d(&tq, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)N, (uint64_t)(K / 8), kWideRows,
-                      kGemmKB / 8, CU_TENSOR_MAP_SWIZZLE_NONE))
+                      C::kWKB * kGemmKB / 8, wswz))
         return AWQ_ERR_CUDA;
     if (cudaFuncSetAttribute(gemm_w4a16_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
