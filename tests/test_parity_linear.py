@@ -139,6 +139,19 @@ def test_gemm_ragged_k_tail(lib):
         assert_linear_close(_run(lib, "gemm", X, dq, G, zp), O.linear(X, q, sc, z, K, G, zp))
 
 
+@pytest.mark.parametrize("M,K,N,G,zp", [
+    (40, 4160, 384, 64, False),   # 65 k-blocks, split K: the last split is one k-block of a 4-block stage
+    (130, 704, 1000, 64, True),   # 256-token tiles, 11 k-blocks in 2 splits: the second ends mid-stage
+])
+def test_gemm_split_k_partial_stage(lib, M, K, N, G, zp):
+    """The 128-channel form loads packed weights 4 k-blocks per copy and splits K on whole
+    copies; a split that ends inside one (K not a multiple of 256) uses part of it."""
+    W = inputs.weights(N, K, 0.02, seed=304 + K)
+    X = inputs.activations(M, K, seed=305 + K)
+    q, sc, z, dq = _packed(W, G, zp)
+    assert_linear_close(_run(lib, "gemm", X, dq, G, zp), O.linear(X, q, sc, z, K, G, zp))
+
+
 def test_gemm_outputs_do_not_spill(lib):
     M, K, N, G = 70, 512, 136, 128
     W = inputs.weights(N, K, seed=304)
