@@ -16,9 +16,10 @@
 //               into a ring whose slots the MMAs free.
 //   warp 1      allocates TMEM; one lane issues 4 tcgen05.mma (K = 16 each) per k-block.
 //   warp 2      TMA producer of the packed weights: tile [128 rows x 32 words] = 4 k-blocks per
-//               stage (whole 128-byte lines per row; 32-byte rows cap the copy rate), 128B-
-//               swizzled, into a ring of its own whose slots the dequantisers free as soon
-//               as they have read the words, so that refilling it never waits for the MMAs.
+//               stage (a whole 128-byte line per row; with one 32-byte row per k-block the
+//               copies landed at about 4 B/cycle per SM), 128B-swizzled, into a ring of its
+//               own whose slots the dequantisers free as soon as they have read the words,
+//               so that refilling it never waits for the MMAs.
 //   warps 3..18 dequantise: thread (row, quarter) turns 16 codes per k-block into fp16
 //               (q - z) * scale16 with mask/magic-number arithmetic, a batch of k-blocks per
 //               iteration, and writes them in the 128B-swizzled K-major layout the MMA
